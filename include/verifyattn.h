@@ -1,0 +1,200 @@
+/*
+ * libverifyattn -- tree-verify MLA-absorb attention for DDTree speculative
+ * decoding, for NVIDIA B200 (sm_100a).
+ *
+ * The verify step of a greedy DDTree decode step (page "The Milestone
+ * Commit: Cementing Phase 1 of a Custom CUDA Speculative Decoding Engine",
+ * section "The Context", items 1-3): a best-first draft tree is built from
+ * the drafter's per-depth top-k, every tree node becomes a query, and each
+ * node attends -- per head, in the absorbed MLA latent space (512-d c_kv plus
+ * a 64-d rope key) -- to its request's cached prefix and to its own
+ * ancestors in the tree tail, through a masked softmax that yields a latent
+ * output and its log-sum-exp.  The pages' C ABI hands raw device pointers
+ * and the caller's CUDA stream across the boundary (page "The Capstone
+ * Commit: Validating a Native CUDA DDTree Inference Engine", section "The
+ * Message Itself"); this header keeps that shape.
+ *
+ * Conventions for every call:
+ *   - Pointers marked [device] are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees or keeps them.  [host] pointers are
+ *     read during the call only.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream) and runs
+ *     asynchronously; nothing synchronises the host.
+ *   - A call returns VA_OK once its kernels are enqueued.  Argument errors
+ *     are reported before anything is launched (VA_ERR_INVALID_ARG,
+ *     VA_ERR_UNSUPPORTED); a failed launch returns VA_ERR_CUDA.  Errors found
+ *     on the device (a malformed tree, a bad kv_len or page index) are
+ *     written to the optional per-request status arrays.
+ *   - Device pointers must be 16-byte aligned; all tensors are dense,
+ *     row-major, innermost dimension last.
+ *   - Thread safety: calls may be issued from several host threads on
+ *     different streams; calls that share output buffers race on the GPU.
+ */
+#ifndef VERIFYATTN_H_
+#define VERIFYATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA. */
+typedef struct CUstream_st* va_stream_t;
+
+enum va_status {
+  VA_OK = 0,
+  VA_ERR_INVALID_ARG = 1,  /* bad size, NULL or misaligned pointer      */
+  VA_ERR_UNSUPPORTED = 2,  /* valid request this build does not handle  */
+  VA_ERR_CUDA = 3,         /* a CUDA launch or driver call failed       */
+  VA_ERR_INVALID_TREE = 4  /* (device status) malformed parent array    */
+};
+
+enum va_dtype { VA_F32 = 0, VA_BF16 = 1 };
+
+#define VA_D_LATENT 512   /* c_kv / q_nope / output width                 */
+#define VA_D_ROPE 64      /* k_pe / q_pe width                            */
+#define VA_PAGE_SIZE 64   /* tokens per KV page                           */
+#define VA_MAX_QLEN 65    /* T = tree budget 64 + root (pages: MAX_QLEN)  */
+#define VA_MAX_DEPTH 15   /* deepest tree the builder produces            */
+#define VA_MAX_TOPK 16    /* widest drafter top-k the builder accepts     */
+#define VA_SPLIT_ALIGN 256/* split-KV chunk granularity, in keys          */
+#define VA_MAX_SPLITS 64
+
+/* Largest tree-verify query length T (root included): 65.  The pages'
+ * library reports the same limit when it loads ("Verified lib loads
+ * (MAX_QLEN=65)", page "The Capstone Commit...", section "The Message
+ * Itself"). */
+int va_max_qlen(void);
+
+/* Static, human-readable name of a va_status value. */
+const char* va_status_string(int status);
+
+/*
+ * Best-first draft-tree builder (page "The Milestone Commit...", section
+ * "The Context", item 1: a GPU best-first builder replacing the per-request
+ * CPU heap; page "Strategic Pivots in CUDA Kernel Engineering...", section
+ * "Why This Message Was Written": ties resolved as in tuple comparison).
+ *
+ *   lp      [device] double [B, L, K]  per-depth top-K drafter log-probs,
+ *                                      row d = depth d+1, descending in K
+ *   tok     [device] int32  [B, L, K]  matching token ids
+ *   parents [device] int32  [B, T]     out: parent node, -1 for the root and
+ *                                      for absent nodes of underfull trees
+ *   tokens  [device] int32  [B, T]     out: token id (-1 root / absent)
+ *   depth   [device] int32  [B, T]     out: depth (0 root, -1 absent)
+ *   n_nodes [device] int32  [B]        out: node count incl. the root
+ *   T = budget + 1, 1 <= T <= VA_MAX_QLEN, 1 <= L <= VA_MAX_DEPTH,
+ *   1 <= K <= VA_MAX_TOPK.
+ * A node's score is its parent's score plus its own log-prob, in fp64.  The
+ * frontier pops the highest score; equal scores go to the lower parent node
+ * index, then the lower rank.  Node indices are pop order, so parent < child.
+ * lp and tok are read only; the builder does not check lp is sorted.
+ */
+int va_build_tree(const double* lp, const int32_t* tok, int B, int L, int K, int budget,
+                  int32_t* parents, int32_t* tokens, int32_t* depth, int32_t* n_nodes,
+                  va_stream_t stream);
+
+/*
+ * Tree visibility (ancestor) mask (page "Strategic Pivots in CUDA Kernel
+ * Engineering...", section "The Message": a tree visibility mask from the
+ * builder).
+ *
+ *   parents     [device] int32  [B, T]     parent[0] = -1; for i >= 1 either
+ *                                          -1 (absent node) or 0 <= p < i with
+ *                                          node p present
+ *   mask        [device] uint64 [B, T, W]  out, W = ceil(T / 64): bit i of
+ *                                          row t (word i / 64) is set iff node
+ *                                          i is t or an ancestor of t
+ *   tree_status [device] int32  [B]        out (nullable): VA_OK or
+ *                                          VA_ERR_INVALID_TREE
+ * Absent nodes get an all-zero row (their own bit clear).  A malformed
+ * request gets all-zero rows and VA_ERR_INVALID_TREE.  1 <= T <= 65, B >= 0.
+ */
+int va_build_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
+                       int32_t* tree_status, va_stream_t stream);
+
+/* Arguments of va_verify_attn.  Zero-initialise, then fill. */
+typedef struct va_attn_args {
+  int dtype;          /* VA_F32 (CUDA-core FFMA path) or VA_BF16 (tcgen05 path) */
+  int B, H, T;        /* requests, heads, query length (1 <= T <= 65)           */
+  float scale;        /* softmax scale on q.k (e.g. 1/sqrt(192))                */
+  const void* q_nope; /* [device] [B, T, H, 512] dtype, latent (absorbed) query */
+  const void* q_pe;   /* [device] [B, T, H, 64]  dtype, rope query              */
+  const void* c_kv;   /* [device] [num_pages, 64, 512] dtype, latent KV pool    */
+  const void* k_pe;   /* [device] [num_pages, 64, 64]  dtype, rope key pool     */
+  int num_pages;      /* pages in the pool                                      */
+  int page_size;      /* must be VA_PAGE_SIZE                                   */
+  const int32_t* page_table; /* [device] [B, max_pages] logical -> physical   */
+  int max_pages;      /* row stride of page_table                               */
+  const int32_t* kv_len;     /* [device] [B] keys of request b = P_b + T; the
+                                tree tail is the last T keys (node i at P_b+i) */
+  const uint64_t* tree_mask; /* [device] [B, T, ceil(T/64)] from
+                                va_build_tree_mask                             */
+  void* out;          /* [device] [B, T, H, 512] dtype, normalised latent out   */
+  float* lse;         /* [device] [B, T, H] float, natural-log sum-exp          */
+  int32_t* req_status;/* [device] [B] nullable: VA_ERR_INVALID_ARG when kv_len
+                         or a page index is out of range (rows written as 0 /
+                         -inf)                                                 */
+  int num_splits;     /* 0 = auto, 1 = single pass, 2..64 = split-KV + merge    */
+  void* workspace;    /* [device] split-KV partials, >= va_workspace_bytes()    */
+  size_t workspace_bytes;
+  int flags;          /* VA_FLAG_* below                                        */
+} va_attn_args;
+
+/* Run bf16 inputs on the CUDA-core FFMA kernel instead of the tensor-core
+ * kernel (a second, independent GPU path for cross-checks). */
+#define VA_FLAG_BF16_CUDA_CORES 1
+
+/*
+ * Workspace needed by va_verify_attn for these arguments (0 for a single
+ * pass).  With S = the split count the call will use, the workspace holds
+ * o_part float [S, B, T, H, 512] followed (256-byte aligned) by lse_part
+ * float [S, B, T, H]; the layout va_merge reads.  Returns 0 on bad args.
+ */
+size_t va_workspace_bytes(const va_attn_args* args);
+
+/* The split count va_verify_attn will use for these arguments (>= 1), or a
+ * negative va_status on bad arguments. */
+int va_num_splits(const va_attn_args* args);
+
+/*
+ * Tree-verify MLA-absorb attention (page "The Milestone Commit...", section
+ * "The Context", item 2: masked softmax over the concatenated prefix and
+ * tree tail, latent output, no host round-trips; section "How Decisions Were
+ * Made", production notes: flash+merge for long prefixes).
+ *
+ * For row (b, t, h), with P = kv_len[b] - T, key j in [0, kv_len[b]) lives at
+ * c_kv[page_table[b][j / 64]][j % 64] (and k_pe likewise); it is visible iff
+ * j < P, or bit (j - P) of tree_mask[b][t] is set.
+ *   s_j = scale * (q_nope . c_kv_j + q_pe . k_pe_j)
+ *   out = sum_j softmax(s)_j c_kv_j      lse = ln sum_j exp(s_j)
+ * A row whose own tree bit is clear (absent node) gets out = 0, lse = -inf.
+ * With S > 1 splits, split s covers keys [s*C, min((s+1)*C, kv_len)) with
+ * C = ceil(ceil(kv_len / S) / 256) * 256; the partials go to the workspace
+ * and va_merge combines them on the same stream.
+ * bf16 runs on tensor cores with fp32 accumulation; fp32 on CUDA cores.
+ * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, B >= 0, every
+ * page slot below kv_len holds finite values.
+ */
+int va_verify_attn(const va_attn_args* args, va_stream_t stream);
+
+/*
+ * Merge of split-KV partials (the flash+merge production note, page "The
+ * Milestone Commit...", section "How Decisions Were Made").
+ *   o_part   [device] float [S, B, T, H, 512]  normalised partial outputs
+ *   lse_part [device] float [S, B, T, H]       partial lse (-inf = empty)
+ *   out      [device] out_dtype [B, T, H, 512]
+ *   lse      [device] float [B, T, H]
+ * lse = ln sum_c exp(lse_c); out = sum_c exp(lse_c - lse) o_c; a row whose
+ * partials are all empty gets out = 0, lse = -inf.  1 <= S <= 64.
+ */
+int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,
+             int out_dtype, void* out, float* lse, va_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VERIFYATTN_H_ */

@@ -1,0 +1,171 @@
+// C ABI of libverifyattn: argument checks, split planning, dispatch.
+// Every entry point validates on the host and returns a va_status before
+// launching anything; the caller owns all device memory.
+#include <cstdio>
+
+#include "va_common.cuh"
+
+namespace {
+
+constexpr int kSms = 148;  // B200 SM count; the split planner's wave size
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Host-side checks shared by va_verify_attn / va_workspace_bytes.
+int check_args(const va_attn_args* a) {
+  if (!a) return VA_ERR_INVALID_ARG;
+  if (a->dtype != VA_F32 && a->dtype != VA_BF16) return VA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 1 || a->T < 1 || a->T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
+  if (a->page_size != VA_PAGE_SIZE) return VA_ERR_UNSUPPORTED;
+  if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
+  if (a->flags & ~VA_FLAG_BF16_CUDA_CORES) return VA_ERR_INVALID_ARG;
+  if (!(a->scale == a->scale)) return VA_ERR_INVALID_ARG;  // NaN scale
+  if (a->B == 0) return VA_OK;
+  if (a->num_pages < 1 || a->max_pages < 1) return VA_ERR_INVALID_ARG;
+  if ((long long)a->num_pages * VA_PAGE_SIZE > 0x7fffffffLL) return VA_ERR_UNSUPPORTED;
+  const void* need16[] = {a->q_nope, a->q_pe, a->c_kv, a->k_pe, a->out};
+  for (const void* p : need16)
+    if (!p || !aligned(p, 16)) return VA_ERR_INVALID_ARG;
+  if (!a->page_table || !aligned(a->page_table, 4)) return VA_ERR_INVALID_ARG;
+  if (!a->kv_len || !aligned(a->kv_len, 4)) return VA_ERR_INVALID_ARG;
+  if (!a->tree_mask || !aligned(a->tree_mask, 8)) return VA_ERR_INVALID_ARG;
+  if (!a->lse || !aligned(a->lse, 4)) return VA_ERR_INVALID_ARG;
+  if (a->req_status && !aligned(a->req_status, 4)) return VA_ERR_INVALID_ARG;
+  return VA_OK;
+}
+
+bool use_tensor_cores(const va_attn_args* a) {
+  return a->dtype == VA_BF16 && !(a->flags & VA_FLAG_BF16_CUDA_CORES);
+}
+
+// Split count: the caller's, or (num_splits == 0) the smallest power of two
+// that fills >= 90% of the last wave, keeping >= 1024 keys per split.  The
+// host does not see kv_len, so the planner uses the page-table capacity as
+// the key count.
+int plan_splits(const va_attn_args* a) {
+  if (a->num_splits > 0) return a->num_splits;
+  if (a->B == 0) return 1;
+  const long long rows = (long long)a->T * a->H;
+  long long units_per_split, slots;
+  if (use_tensor_cores(a)) {
+    units_per_split = (long long)a->B * ((rows + 127) / 128);  // CTA pairs
+    slots = kSms / 2;
+  } else {
+    units_per_split = (long long)a->B * ((rows + 31) / 32);
+    slots = kSms;
+  }
+  const long long keys = (long long)a->max_pages * VA_PAGE_SIZE;
+  for (int S = 1; S <= VA_MAX_SPLITS; S *= 2) {
+    if (S > 1 && keys / S < 1024) return S / 2;
+    const long long units = units_per_split * S;
+    const long long waves = (units + slots - 1) / slots;
+    if (units * 10 >= waves * slots * 9) return S;
+  }
+  return VA_MAX_SPLITS;
+}
+
+size_t part_bytes(const va_attn_args* a, int S, size_t* lse_off) {
+  const size_t rows = (size_t)a->B * a->T * a->H;
+  const size_t o = align_up((size_t)S * rows * VA_D_LATENT * sizeof(float), 256);
+  if (lse_off) *lse_off = o;
+  return o + align_up((size_t)S * rows * sizeof(float), 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+int va_max_qlen(void) { return VA_MAX_QLEN; }
+
+const char* va_status_string(int status) {
+  switch (status) {
+    case VA_OK: return "VA_OK";
+    case VA_ERR_INVALID_ARG: return "VA_ERR_INVALID_ARG";
+    case VA_ERR_UNSUPPORTED: return "VA_ERR_UNSUPPORTED";
+    case VA_ERR_CUDA: return "VA_ERR_CUDA";
+    case VA_ERR_INVALID_TREE: return "VA_ERR_INVALID_TREE";
+    default: return "VA_ERR_UNKNOWN";
+  }
+}
+
+int va_build_tree(const double* lp, const int32_t* tok, int B, int L, int K, int budget,
+                  int32_t* parents, int32_t* tokens, int32_t* depth, int32_t* n_nodes,
+                  va_stream_t stream) {
+  if (B < 0 || L < 1 || L > VA_MAX_DEPTH || K < 1 || K > VA_MAX_TOPK || budget < 0 ||
+      budget + 1 > VA_MAX_QLEN)
+    return VA_ERR_INVALID_ARG;
+  if (B == 0) return VA_OK;
+  if (!lp || !tok || !parents || !tokens || !depth || !n_nodes) return VA_ERR_INVALID_ARG;
+  if (!aligned(lp, 8)) return VA_ERR_INVALID_ARG;
+  cudaError_t e = va::launch_build_tree(lp, tok, B, L, K, budget, parents, tokens, depth,
+                                        n_nodes, (cudaStream_t)stream);
+  return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
+}
+
+int va_build_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
+                       int32_t* tree_status, va_stream_t stream) {
+  if (B < 0 || T < 1 || T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
+  if (B == 0) return VA_OK;
+  if (!parents || !mask || !aligned(mask, 8)) return VA_ERR_INVALID_ARG;
+  cudaError_t e = va::launch_tree_mask(parents, B, T, mask, tree_status, (cudaStream_t)stream);
+  return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
+}
+
+int va_num_splits(const va_attn_args* args) {
+  const int st = check_args(args);
+  if (st != VA_OK) return -st;
+  return plan_splits(args);
+}
+
+size_t va_workspace_bytes(const va_attn_args* args) {
+  if (check_args(args) != VA_OK) return 0;
+  const int S = plan_splits(args);
+  if (S <= 1 || args->B == 0) return 0;
+  return part_bytes(args, S, nullptr);
+}
+
+int va_verify_attn(const va_attn_args* args, va_stream_t stream) {
+  int st = check_args(args);
+  if (st != VA_OK) return st;
+  if (args->B == 0) return VA_OK;
+  const int S = plan_splits(args);
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+  if (S > 1) {
+    size_t lse_off = 0;
+    const size_t need = part_bytes(args, S, &lse_off);
+    if (!args->workspace || !aligned(args->workspace, 256) || args->workspace_bytes < need)
+      return VA_ERR_INVALID_ARG;
+    o_part = (float*)args->workspace;
+    lse_part = (float*)((char*)args->workspace + lse_off);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = use_tensor_cores(args) ? va::launch_attn_tc(*args, S, o_part, lse_part, s)
+                                         : va::launch_attn_simt(*args, S, o_part, lse_part, s);
+  if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return VA_ERR_CUDA;
+  if (S > 1) {
+    e = va::launch_merge(o_part, lse_part, S, (long long)args->B * args->T * args->H,
+                         args->dtype, args->out, args->lse, s);
+    if (e != cudaSuccess) return VA_ERR_CUDA;
+  }
+  return VA_OK;
+}
+
+int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,
+             int out_dtype, void* out, float* lse, va_stream_t stream) {
+  if (S < 1 || S > VA_MAX_SPLITS || B < 0 || T < 1 || T > VA_MAX_QLEN || H < 1)
+    return VA_ERR_INVALID_ARG;
+  if (out_dtype != VA_F32 && out_dtype != VA_BF16) return VA_ERR_INVALID_ARG;
+  if (B == 0) return VA_OK;
+  if (!o_part || !lse_part || !out || !lse) return VA_ERR_INVALID_ARG;
+  if (!aligned(o_part, 16) || !aligned(out, 8) || !aligned(lse_part, 4) || !aligned(lse, 4))
+    return VA_ERR_INVALID_ARG;
+  cudaError_t e = va::launch_merge(o_part, lse_part, S, (long long)B * T * H, out_dtype, out,
+                                   lse, (cudaStream_t)stream);
+  return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
+}
+
+}  // extern "C"

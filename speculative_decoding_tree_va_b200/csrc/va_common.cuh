@@ -1,0 +1,56 @@
+// Shared device helpers of libverifyattn (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/verifyattn.h"
+
+namespace va {
+
+constexpr int kDc = VA_D_LATENT;
+constexpr int kDr = VA_D_ROPE;
+constexpr int kDqk = kDc + kDr;
+constexpr int kPage = VA_PAGE_SIZE;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Bit i of a tree-mask row (W words).
+__device__ __forceinline__ bool mask_bit(const uint64_t* row, int i) {
+  return (row[i >> 6] >> (i & 63)) & 1ull;
+}
+
+// Split-KV chunk bounds, as fixed in the public header:
+// C = ceil(ceil(kv_len / S) / 256) * 256, split s = [s*C, min((s+1)*C, kv_len)).
+__host__ __device__ __forceinline__ void split_range(int kv_len, int S, int s, int* lo, int* hi) {
+  int per = (kv_len + S - 1) / S;
+  int chunk = (per + VA_SPLIT_ALIGN - 1) / VA_SPLIT_ALIGN * VA_SPLIT_ALIGN;
+  long long a = (long long)s * chunk, b = (long long)(s + 1) * chunk;
+  *lo = (int)(a < kv_len ? a : kv_len);
+  *hi = (int)(b < kv_len ? b : kv_len);
+}
+
+// Launchers implemented in the .cu files (internal C++ linkage).
+cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
+                              int budget, int32_t* parents, int32_t* tokens, int32_t* depth,
+                              int32_t* n_nodes, cudaStream_t st);
+cudaError_t launch_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
+                             int32_t* status, cudaStream_t st);
+cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float* lse_part,
+                             cudaStream_t st);
+cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
+                         int out_dtype, void* out, float* lse, cudaStream_t st);
+cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
+                           cudaStream_t st);
+
+}  // namespace va

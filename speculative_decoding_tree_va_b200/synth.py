@@ -82,11 +82,11 @@ WORKLOAD_ORDER = ["fp32-tiny", "fp32-page-test", "bf16-deep", "bf16-b64-ragged",
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (nearest, ties to even); returns uint16 bit patterns.
 
-    Inputs are finite N(0,1) draws, so no NaN handling is needed here.
+    Inputs are finite draws, so the 32-bit sum cannot wrap (only NaN bit
+    patterns lie within 0x8000 of 2^32) and no NaN handling is needed.
     """
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + (0x7FFF + ((u >> 16) & 1))) >> 16).astype(np.uint16)
 
 
 def bf16_to_f32(u: np.ndarray) -> np.ndarray:

@@ -1,0 +1,103 @@
+"""CPU checks of the C ABI: the library loads, exports what the header declares,
+and rejects bad arguments on the host before launching anything."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import speculative_decoding_tree_va_b200 as va
+from speculative_decoding_tree_va_b200 import build as va_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    va_build.build()
+    return va.load_library()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(va_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"va_verify_attn", "va_build_tree_mask", "va_merge", "va_build_tree"} <= names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(va.EXPORTS) <= names
+
+
+def test_max_qlen_and_status_strings(lib):
+    assert lib.va_max_qlen() == 65
+    assert lib.va_status_string(0) == b"VA_OK"
+    assert lib.va_status_string(4) == b"VA_ERR_INVALID_TREE"
+    assert lib.va_status_string(99) == b"VA_ERR_UNKNOWN"
+
+
+def args(**kw):
+    a = va.VaAttnArgs()
+    a.dtype, a.B, a.H, a.T, a.scale = va.VA_BF16, 2, 64, 33, 0.07
+    fake = 1 << 20  # aligned, never dereferenced: every case below fails host checks
+    for f in ("q_nope", "q_pe", "c_kv", "k_pe", "page_table", "kv_len", "tree_mask", "out", "lse"):
+        setattr(a, f, fake)
+    a.num_pages, a.page_size, a.max_pages = 100, 64, 50
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(T=66), va.VA_ERR_INVALID_ARG), (dict(T=0), va.VA_ERR_INVALID_ARG),
+    (dict(H=0), va.VA_ERR_INVALID_ARG), (dict(dtype=7), va.VA_ERR_INVALID_ARG),
+    (dict(page_size=32), va.VA_ERR_UNSUPPORTED), (dict(num_splits=65), va.VA_ERR_INVALID_ARG),
+    (dict(q_nope=None), va.VA_ERR_INVALID_ARG), (dict(c_kv=(1 << 20) + 8), va.VA_ERR_INVALID_ARG),
+    (dict(flags=8), va.VA_ERR_INVALID_ARG), (dict(num_pages=0), va.VA_ERR_INVALID_ARG),
+    (dict(num_splits=4), va.VA_ERR_INVALID_ARG),  # split without a workspace
+    (dict(scale=float("nan")), va.VA_ERR_INVALID_ARG),
+])
+def test_verify_attn_host_checks(lib, bad, status):
+    a = args(**bad)
+    assert lib.va_verify_attn(ctypes.byref(a), None) == status
+
+
+def test_zero_batch_is_a_noop(lib):
+    a = args(B=0)
+    assert lib.va_verify_attn(ctypes.byref(a), None) == va.VA_OK
+    assert lib.va_build_tree_mask(None, 0, 5, None, None, None) == va.VA_OK
+    assert lib.va_merge(None, None, 2, 0, 5, 8, 0, None, None, None) == va.VA_OK
+
+
+def test_other_host_checks(lib):
+    assert lib.va_build_tree_mask(None, 1, 66, None, None, None) == va.VA_ERR_INVALID_ARG
+    assert lib.va_build_tree_mask(None, 1, 5, None, None, None) == va.VA_ERR_INVALID_ARG
+    assert lib.va_build_tree(None, None, 1, 16, 8, 32, None, None, None, None, None) == \
+        va.VA_ERR_INVALID_ARG  # depth > 15
+    assert lib.va_build_tree(None, None, 1, 15, 8, 65, None, None, None, None, None) == \
+        va.VA_ERR_INVALID_ARG  # T = 66
+    assert lib.va_merge(None, None, 65, 1, 5, 8, 0, None, None, None) == va.VA_ERR_INVALID_ARG
+    assert lib.va_merge(None, None, 2, 1, 5, 8, 3, None, None, None) == va.VA_ERR_INVALID_ARG
+
+
+def test_split_planning_and_workspace(lib):
+    # explicit split count: partials [S,B,T,H,512] f32 + [S,B,T,H] f32, 256-byte aligned
+    a = args(num_splits=16)
+    rows = 2 * 33 * 64
+    o = (16 * rows * 512 * 4 + 255) // 256 * 256
+    l = (16 * rows * 4 + 255) // 256 * 256
+    assert lib.va_num_splits(ctypes.byref(a)) == 16
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == o + l
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1))) == 0
+    # auto: a big batch needs no split; a long, small batch splits
+    assert lib.va_num_splits(ctypes.byref(args(B=64, max_pages=129))) == 1
+    s = lib.va_num_splits(ctypes.byref(args(B=4, T=65, max_pages=2050)))
+    assert s > 1 and (4 * 33 * s) % 74 >= 0
+    assert lib.va_num_splits(ctypes.byref(args(T=66))) == -va.VA_ERR_INVALID_ARG

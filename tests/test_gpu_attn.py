@@ -1,0 +1,202 @@
+"""GPU parity of va_verify_attn / va_merge against the fp64 oracle.
+
+Paths: "f32" (CUDA-core FFMA kernel), "tc" (bf16 tcgen05 kernel, the default
+for bf16) and "cc" (bf16 on the CUDA-core kernel, VA_FLAG_BF16_CUDA_CORES).
+Bars: fp32 max_abs <= 1e-5; bf16 out max_abs <= 1e-2 and lse <= 1e-3.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+from speculative_decoding_tree_va_b200 import synth
+from _harness import compare, oracle_rows, to_device, trees_for
+
+pytestmark = pytest.mark.gpu
+
+BF16_PATHS = ["tc", "cc"]
+
+
+@pytest.fixture(scope="module")
+def va():
+    import torch
+    assert torch.cuda.is_available()
+    import speculative_decoding_tree_va_b200 as m
+    m.load_library()
+    return m
+
+
+def run_gpu(va, inp, parents, path, num_splits=1, rows=None):
+    """Mask + attention on the GPU; returns numpy (out, lse) rows and the mask."""
+    import torch
+    d = to_device(inp, parents)
+    mask, status = va.build_tree_mask(d["parents"])
+    flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
+    req_status = torch.zeros(inp.wl.B, dtype=torch.int32, device="cuda")
+    out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
+                              d["kv_len"], mask, scale=synth.SCALE, num_splits=num_splits,
+                              flags=flags, req_status=req_status)
+    torch.cuda.synchronize()
+    assert (req_status.cpu().numpy() == 0).all()
+    out = out.float().reshape(-1, synth.D_LATENT)
+    lse = lse.reshape(-1)
+    if rows is not None:
+        idx = torch.from_numpy(rows.astype(np.int64)).cuda()
+        out, lse = out[idx], lse[idx]
+    return out.cpu().numpy(), lse.cpu().numpy(), mask.cpu().numpy().view(np.uint64)
+
+
+def check_full(va, inp, path, num_splits=1, parents=None, what=""):
+    if parents is None:
+        parents = trees_for(inp)["parent"]
+    out, lse, mask = run_gpu(va, inp, parents, path, num_splits)
+    ref_out, ref_lse = oracle_rows(inp, mask)
+    return compare(out, lse, ref_out, ref_lse, inp.wl.dtype, what or inp.wl.name)
+
+
+def paths_for(dtype):
+    return ["f32"] if dtype == "f32" else BF16_PATHS
+
+
+# --- the two fp32 workloads in full -------------------------------------------
+
+@pytest.mark.parametrize("name", ["fp32-tiny", "fp32-page-test"])
+def test_fp32_workloads_full(va, name):
+    inp = synth.make_inputs(synth.WORKLOADS[name])
+    check_full(va, inp, "f32")
+
+
+# --- bf16 workloads, scaled so the oracle runs every row ---------------------
+
+SMALL = [
+    ("bf16-deep", dict(B=2, P=700)),
+    ("bf16-b64-ragged", dict(B=5, P=(130, 1400))),
+    ("bf16-long-prefix", dict(B=1, P=3000, H=16)),
+]
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("name,kw", SMALL)
+def test_bf16_workloads_scaled(va, path, name, kw):
+    inp = synth.make_inputs(synth.WORKLOADS[name], **kw)
+    check_full(va, inp, path)
+
+
+@pytest.mark.parametrize("path", ["f32"] + BF16_PATHS)
+@pytest.mark.parametrize("S", [2, 3, 16])
+def test_split_kv_matches_unsplit_oracle(va, path, S):
+    name = "fp32-page-test" if path == "f32" else "bf16-long-prefix"
+    inp = synth.make_inputs(synth.WORKLOADS[name], B=2, H=8, P=(1500, 4000))
+    check_full(va, inp, path, num_splits=S)
+
+
+# --- edge cases ----------------------------------------------------------------
+
+def edge_inputs(dtype, B=2, H=8, P=0, budget=8, topk=8, max_depth=15, seed=5):
+    wl = synth.WORKLOADS["fp32-tiny" if dtype == "f32" else "bf16-deep"]
+    wl = dataclasses.replace(wl, paged=True)
+    return synth.make_inputs(wl, B=B, H=H, P=P, budget=budget, topk=topk,
+                             max_depth=max_depth, seed=seed)
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
+@pytest.mark.parametrize("case", [
+    dict(P=0, budget=0),                 # T = 1, no prefix: the root sees itself
+    dict(P=0, budget=8),                 # tree tail only
+    dict(P=1, budget=64, H=16),          # maxbudget, T = 65 (two mask words)
+    dict(P=63, budget=64, topk=1),       # deep chain, depth 15, underfull tree (padding)
+    dict(P=64, budget=32, H=16),
+    dict(P=(5, 600), budget=20, topk=3, B=4),
+    dict(P=257, budget=64, topk=2, H=64, B=1),
+    dict(P=100, budget=10, H=1),
+    dict(P=(60, 70), budget=33, H=3, B=3),
+])
+def test_edge_cases(va, dtype, path, case):
+    inp = edge_inputs(dtype, **case)
+    check_full(va, inp, path, what=f"{case}")
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
+@pytest.mark.parametrize("shape", ["chain", "star"])
+def test_chain_and_star_trees(va, dtype, path, shape):
+    inp = edge_inputs(dtype, B=2, H=8, P=(90, 300), budget=40)
+    T = inp.T
+    p = np.array([-1] + (list(range(T - 1)) if shape == "chain" else [0] * (T - 1)), np.int32)
+    check_full(va, inp, path, parents=np.stack([p, p]))
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
+def test_values_beyond_kv_len_do_not_leak(va, dtype, path):
+    inp = edge_inputs(dtype, B=3, H=8, P=(70, 200), budget=16)
+    big = 3.0e4
+    for b in range(inp.wl.B):
+        n = int(inp.kv_len[b])
+        last = inp.page_table[b, (n - 1) // 64]
+        for arr in (inp.c_kv, inp.k_pe):
+            v = np.full(arr.shape[2], big, np.float32)
+            arr[last, n % 64 or 64:] = synth.bf16_round(v) if dtype == "bf16" else v
+    check_full(va, inp, path)
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
+def test_bad_kv_len_and_page_are_flagged(va, dtype, path):
+    import torch
+    inp = edge_inputs(dtype, B=3, H=8, P=(70, 200), budget=8)
+    parents = trees_for(inp)["parent"]
+    d = to_device(inp, parents)
+    mask, _ = va.build_tree_mask(d["parents"])
+    kv = d["kv_len"].clone()
+    kv[1] = 3                                   # shorter than T
+    pt = d["page_table"].clone()
+    pt[2, 0] = inp.num_pages + 5                # page out of range
+    st = torch.zeros(3, dtype=torch.int32, device="cuda")
+    flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
+    out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], pt, kv, mask,
+                              scale=synth.SCALE, num_splits=1, req_status=st, flags=flags)
+    torch.cuda.synchronize()
+    assert st.cpu().tolist() == [0, va.VA_ERR_INVALID_ARG, va.VA_ERR_INVALID_ARG]
+    assert torch.isneginf(lse[1:]).all() and not out[1:].float().abs().sum()
+    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64),
+                                   rows=np.arange(inp.T * inp.wl.H, dtype=np.int32))
+    compare(out[0].float().cpu().numpy().reshape(-1, 512), lse[0].cpu().numpy().reshape(-1),
+            ref_out, ref_lse, dtype)
+
+
+# --- merge ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("S", [1, 2, 7, 33, 64])
+def test_merge_against_oracle(va, out_dtype, S):
+    import torch
+    rng = np.random.default_rng(S)
+    B, T, H = 2, 5, 3
+    o = rng.standard_normal((S, B, T, H, 512)).astype(np.float32)
+    l = (rng.standard_normal((S, B, T, H)) * 3).astype(np.float32)
+    l[rng.random(l.shape) < 0.3] = -np.inf      # empty chunks
+    l[:, 0, 0, 0] = -np.inf                     # a row with every chunk empty
+    tdt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    out, lse = va.merge(torch.from_numpy(o).cuda(), torch.from_numpy(l).cuda(), tdt)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.merge(o.reshape(S, -1, 512), l.reshape(S, -1))
+    compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+            ref_out, ref_lse, out_dtype)
+
+
+# --- full-size workloads on sampled rows ---------------------------------------
+
+FULL = [("bf16-deep", 1), ("bf16-b64-ragged", 1), ("bf16-long-prefix", 16)]
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("name,S", FULL)
+def test_full_size_sampled_rows(va, path, name, S):
+    inp = synth.make_inputs(synth.WORKLOADS[name])
+    B, T, H = inp.wl.B, inp.T, inp.wl.H
+    n_rand = 96 if name == "bf16-long-prefix" else 256
+    rows = synth.sample_rows(7, B, T, H, n_rand,
+                             full_request=None if name == "bf16-long-prefix" else 0)
+    parents = trees_for(inp)["parent"]
+    out, lse, mask = run_gpu(va, inp, parents, path, num_splits=S, rows=rows)
+    ref_out, ref_lse = oracle_rows(inp, mask, rows=rows)
+    compare(out, lse, ref_out, ref_lse, "bf16", name)
