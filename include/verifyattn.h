@@ -193,6 +193,14 @@ int va_verify_attn(const va_attn_args* args, va_stream_t stream);
 int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,
              int out_dtype, void* out, float* lse, va_stream_t stream);
 
+/*
+ * Diagnostic: number of bounded barrier waits inside the tensor-core kernel
+ * that expired on the current device since the library was loaded (each
+ * expiry also flags its request with VA_ERR_CUDA).  Synchronises the
+ * device; returns 0xFFFFFFFF if the counter cannot be read.
+ */
+unsigned int va_device_timeouts(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,8 @@ VA_FLAG_BF16_CUDA_CORES = 1
 D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",
-           "va_workspace_bytes", "va_num_splits", "va_verify_attn", "va_merge")
+           "va_workspace_bytes", "va_num_splits", "va_verify_attn", "va_merge",
+           "va_device_timeouts")
 
 
 class VaAttnArgs(ctypes.Structure):
@@ -74,6 +75,7 @@ def load_library(path: Optional[str] = None):
     lib.va_verify_attn.restype = I
     lib.va_merge.argtypes = [V, V, I, I, I, I, I, V, V, V]
     lib.va_merge.restype = I
+    lib.va_device_timeouts.argtypes, lib.va_device_timeouts.restype = [], ctypes.c_uint
     if path is None:
         _lib = lib
     return lib
@@ -97,6 +99,11 @@ def _ptr(t):
 
 def max_qlen() -> int:
     return load_library().va_max_qlen()
+
+
+def device_timeouts() -> int:
+    """Expired bounded waits in the tensor-core kernel since load (synchronises)."""
+    return int(load_library().va_device_timeouts())
 
 
 def build_tree(lp, tok, budget: int, stream=None):

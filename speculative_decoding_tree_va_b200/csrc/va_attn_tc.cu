@@ -1,9 +1,670 @@
-// Tensor-core (tcgen05) bf16 tree-verify attention -- placeholder until the
-// sm_100a kernel lands; reports "not supported" so no silent fallback exists.
+// Tensor-core (tcgen05) bf16 tree-verify MLA-absorb attention for sm_100a.
+//
+// What it computes (page "The Milestone Commit...", section "The Context",
+// item 2; MLA absorb from section "Input Knowledge Required"): for every
+// tree-node query row, a masked softmax over the request's paged prefix and
+// the row's ancestors in the tree tail, in the 512-d latent space plus the
+// 64-d rope key, giving the normalised latent output and its log-sum-exp.
+// The flash-decode split for long prefixes (section "How Decisions Were
+// Made", production notes) is a grid dimension; va_merge combines splits.
+//
+// Design (B200-native; the pages' block-per-(batch, head, query) kernel for
+// sm_120 is not used):
+//  * All H*T query rows of a request share each key, so QK^T and PV are
+//    dense bf16 contractions on the 5th-gen tensor cores.  A 64-row x 512
+//    fp32 output accumulator is 128 KB, half of one SM's tensor memory, so
+//    a CTA pair (cluster of 2) runs tcgen05.mma.cta_group::2 with M = 128:
+//    each CTA holds 64 query rows, and the pair splits every B operand.
+//  * Key tiles of 256 keys (4 pages).  QK: N = 256 keys, CTA r supplies keys
+//    [128r, 128r+128).  PV: two MMAs of N = 256 latent columns; CTA r
+//    supplies columns [256c + 128r, +128) of chunk c.  TMEM per CTA:
+//    S0 | S1 (128 columns each, double-buffered scores) | O (256 columns).
+//  * Data arrives by TMA (128-byte swizzle) into a ring of 16 KB slots,
+//    page-table indexed, one 64-token page per box; pages past the request
+//    are addressed out of bounds and read as zeros.
+//  * Warp roles: warp 0 TMA producer, warp 1 MMA issuer (leader CTA only),
+//    warps 2-5 softmax + epilogue.  The MMA order QK(i+1) before PV(i) lets
+//    the softmax of tile i overlap the tensor core.
+//  * Online softmax in the log2 domain.  The running max is only moved (and
+//    O rescaled in TMEM) when a tile raises it by more than 2^8; otherwise
+//    probabilities up to 2^8 go through bf16/fp32 unchanged (exact maths,
+//    fewer TMEM round trips).  The tree mask is applied only on tiles that
+//    reach the tree tail or the end of the key range.
+//  * Every barrier wait is bounded (1 s): on expiry the CTA sets an abort
+//    flag, every later wait returns at once, and the request is flagged.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "va_common.cuh"
 
 namespace va {
-cudaError_t launch_attn_tc(const va_attn_args&, int, float*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+__device__ unsigned int g_tc_timeouts = 0;  // count of barrier waits that expired
+
+namespace {
+
+constexpr int kThreads = 192;          // 6 warps
+constexpr int kRing = 7;               // KV ring slots
+constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
+constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
+constexpr int kQBytes = 9 * kChunkBytes;   // 64 rows x 576
+constexpr int kPBytes = 4 * kChunkBytes;   // 64 rows x 256 keys
+constexpr int kTileKeys = 256;
+constexpr int kTmemS1 = 128, kTmemO = 256;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr unsigned long long kTimeoutNs = 1000000000ull;
+
+struct TcParams {
+  const int32_t* page_table;
+  const int32_t* kv_len;
+  const uint64_t* tree_mask;
+  void* out;
+  float* lse;
+  float* o_part;
+  float* lse_part;
+  int32_t* req_status;
+  int B, H, T, R, max_pages, num_pages, S;
+  float scale_log2;
+};
+
+struct __align__(16) Ctl {
+  uint64_t full[kRing];
+  uint64_t empty[kRing];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_ready;
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort;
+  int bad_page;
+  float xmax[2][2][64];  // [tile parity][column half][row]
+  float xsum[2][64];
+};
+
+constexpr size_t kSmemBytes = 1024 + kQBytes + kPBytes + (size_t)kRing * kSlotBytes + sizeof(Ctl);
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait on phase `parity` of a local barrier.  Returns false (and
+// marks the CTA aborted) if it did not complete within kTimeoutNs.
+__device__ __noinline__ bool mbar_wait(uint64_t* barp, uint32_t parity, volatile int* abort) {
+  const uint32_t bar = smem_u32(barp);
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int k = 0; k < 32; ++k)
+      if (mbar_try(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kTimeoutNs) {
+      *abort = 1;
+      atomicAdd(&g_tc_timeouts, 1u);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar_cluster, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+               ::"r"(bar_cluster), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+               ::"r"(bar_cluster) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory, completion counted on the
+// pair leader's barrier (cta_group::2 form).  No cluster multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map,
+                                            uint32_t bar_leader, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_leader), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem], issued once for the CTA pair.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrive (once) on the same barrier offset in both CTAs of the pair when all
+// previously issued MMAs of this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)), "h"((uint16_t)0x3) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+        "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
+// version bits = 1.  lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// -------------------------------------------------------------------- kernel
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qp,
+               const __grid_constant__ CUtensorMap tm_ckv,
+               const __grid_constant__ CUtensorMap tm_kpe, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = base;
+  uint8_t* sP = sQ + kQBytes;
+  uint8_t* sRing = sP + kPBytes;
+  Ctl& c = *reinterpret_cast<Ctl*>(sRing + (size_t)kRing * kSlotBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int b = blockIdx.y;
+  const int split = blockIdx.z;
+  const int tile_m = blockIdx.x >> 1;
+  const int row0 = tile_m * 128 + (int)rank * 64;  // first query row of this CTA
+
+  const int kv_len = p.kv_len[b];
+  const bool req_ok = kv_len >= p.T && kv_len <= p.max_pages * kPage;
+  int lo = 0, hi = 0;
+  if (req_ok) split_range(kv_len, p.S, split, &lo, &hi);
+  const int P = kv_len - p.T;
+  const int ntiles = hi > lo ? (hi - lo + kTileKeys - 1) / kTileKeys : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRing; ++s) { mbar_init(&c.full[s], 1); mbar_init(&c.empty[s], 1); }
+    mbar_init(&c.q_full, 1);
+    mbar_init(&c.s_full[0], 1);
+    mbar_init(&c.s_full[1], 1);
+    mbar_init(&c.p_ready, 8);  // 4 softmax warps x 2 CTAs
+    mbar_init(&c.o_done, 1);
+    c.abort = 0;
+    c.bad_page = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;"
+                 ::"r"(smem_u32(&c.tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  volatile int* abort = &c.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      const uint32_t q_bar = map_to_rank(smem_u32(&c.q_full), 0);
+      if (rank == 0) mbar_arrive_expect_tx(q_bar, 2 * kQBytes);
+      const int qrow = b * p.R + row0;
+      for (int ch = 0; ch < 8; ++ch)
+        tma_load_2d(smem_u32(sQ + ch * kChunkBytes), &tm_qn, q_bar, ch * 64, qrow);
+      tma_load_2d(smem_u32(sQ + 8 * kChunkBytes), &tm_qp, q_bar, 0, qrow);
+
+      const int npages_valid = (kv_len + kPage - 1) / kPage;
+      const int oob_row = p.num_pages * kPage;  // first row past the pool: zero fill
+      auto page_row = [&](int pg) -> int {  // logical page -> first pool row
+        if (pg >= npages_valid) return oob_row;
+        const int ph = p.page_table[(size_t)b * p.max_pages + pg];
+        if (ph < 0 || ph >= p.num_pages) return oob_row;  // flagged by the page scan
+        return ph * kPage;
+      };
+      int slot = 0;
+      uint32_t phase = 0;
+      auto acquire = [&]() -> uint32_t {  // wait for a free slot, post the byte count
+        mbar_wait(&c.empty[slot], phase ^ 1, abort);
+        const uint32_t bar = map_to_rank(smem_u32(&c.full[slot]), 0);
+        if (rank == 0) mbar_arrive_expect_tx(bar, 2 * kSlotBytes);
+        return bar;
+      };
+      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
+      auto load_k = [&](int t) {
+        const int kb = lo + t * kTileKeys;
+        const int r0 = page_row(kb / kPage + 2 * (int)rank);
+        const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
+        for (int kc = 0; kc < 9; ++kc) {
+          const uint32_t bar = acquire();
+          const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+          const CUtensorMap* m = kc < 8 ? &tm_ckv : &tm_kpe;
+          const int x = kc < 8 ? kc * 64 : 0;
+          tma_load_2d(dst, m, bar, x, r0);
+          tma_load_2d(dst + kChunkBytes, m, bar, x, r1);
+          advance();
+        }
+      };
+      auto load_v = [&](int t) {
+        const int kb = lo + t * kTileKeys;
+        for (int pg = 0; pg < 4; ++pg) {
+          if (kb + pg * kPage >= hi) break;
+          const int r = page_row(kb / kPage + pg);
+          for (int nc = 0; nc < 2; ++nc) {
+            const uint32_t bar = acquire();
+            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+            const int x = nc * 256 + (int)rank * 128;
+            tma_load_2d(dst, &tm_ckv, bar, x, r);
+            tma_load_2d(dst + kChunkBytes, &tm_ckv, bar, x + 64, r);
+            advance();
+          }
+        }
+      };
+      for (int t = 0; t < ntiles; ++t) {
+        load_k(t);
+        if (t > 0) load_v(t - 1);
+      }
+      load_v(ntiles - 1);
+      // drain: every slot's last load must be consumed before the CTA may exit
+      for (int s = 0; s < kRing; ++s) {
+        mbar_wait(&c.empty[slot], phase ^ 1, abort);
+        advance();
+      }
+    } else if (lane > 0 && ntiles > 0) {
+      // the other 31 lanes check every page index this split reads
+      int bad = 0;
+      for (int pg = lo / kPage + lane - 1; pg < (hi + kPage - 1) / kPage; pg += 31) {
+        const int ph = p.page_table[(size_t)b * p.max_pages + pg];
+        bad |= (ph < 0 || ph >= p.num_pages);
+      }
+      if (bad) c.bad_page = 1;
+    }
+    __syncwarp();
+    named_arrive(2, 160);  // publishes bad_page to the epilogue
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (rank == 0 && lane == 0 && ntiles > 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
+      const uint32_t sq = smem_u32(sQ), sp = smem_u32(sP), sr = smem_u32(sRing);
+      int slot = 0;
+      uint32_t phase = 0;
+      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
+      mbar_wait(&c.q_full, 0, abort);
+      auto qk = [&](int t) {
+        const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
+        for (int kc = 0; kc < 9; ++kc) {
+          mbar_wait(&c.full[slot], phase, abort);
+          tc_fence_after();
+          const uint32_t kslot = sr + slot * kSlotBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = sw128_desc(sq + kc * kChunkBytes + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(kslot + kk * 32, 16, 1024);
+            mma_bf16_pair(d, a, bd, kIdQK, (kc | kk) != 0);
+          }
+          mma_commit_pair(&c.empty[slot]);
+          advance();
+        }
+        mma_commit_pair(&c.s_full[t & 1]);
+      };
+      auto pv = [&](int t) {
+        const int kb = lo + t * kTileKeys;
+        mbar_wait(&c.p_ready, t & 1, abort);
+        tc_fence_after();
+        for (int pg = 0; pg < 4; ++pg) {
+          if (kb + pg * kPage >= hi) break;
+          for (int nc = 0; nc < 2; ++nc) {
+            mbar_wait(&c.full[slot], phase, abort);
+            tc_fence_after();
+            const uint32_t vslot = sr + slot * kSlotBytes;
+            const uint32_t d = tmem + kTmemO + nc * 128;
+            for (int kk = 0; kk < 4; ++kk) {
+              const int k0 = kb + pg * kPage + kk * 16;
+              if (k0 >= hi) break;
+              const int ks = pg * 4 + kk;  // 16-key step inside the 256-key tile
+              const uint64_t a = sw128_desc(sp + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(vslot + kk * 2048, kChunkBytes, 1024);
+              mma_bf16_pair(d, a, bd, kIdPV, !(t == 0 && pg == 0 && kk == 0));
+            }
+            mma_commit_pair(&c.empty[slot]);
+            advance();
+          }
+        }
+        mma_commit_pair(&c.o_done);
+      };
+      for (int t = 0; t < ntiles; ++t) {
+        qk(t);
+        if (t > 0) pv(t - 1);
+      }
+      pv(ntiles - 1);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int q = warp & 3;            // TMEM lane quadrant of this warp
+    const int m = 32 * (q & 1) + lane;  // row within the CTA
+    const int h = q >> 1;              // column half: keys [128h, +128) of each tile
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int row = row0 + m;
+    const bool row_in = row < p.R;
+    const int W = (p.T + 63) >> 6;
+    uint64_t mw0 = 0, mw1 = 0;
+    bool live = false;
+    if (row_in && req_ok) {
+      const int t = row / p.H;
+      const uint64_t* mrow = p.tree_mask + ((size_t)b * p.T + t) * W;
+      mw0 = mrow[0];
+      mw1 = W > 1 ? mrow[1] : 0ull;
+      live = mask_bit(mrow, t);
+    }
+    const uint32_t p_ready_leader = map_to_rank(smem_u32(&c.p_ready), 0);
+    float m_used = -INFINITY, l = 0.f;
+
+    for (int t = 0; t < ntiles; ++t) {
+      const int kb = lo + t * kTileKeys;
+      const int j0 = kb + 128 * h;  // key of this thread's first column
+      mbar_wait(&c.s_full[t & 1], (t >> 1) & 1, abort);
+      tc_fence_after();
+      float x[128];
+      const uint32_t s_addr = tmem + lane_base + ((t & 1) ? kTmemS1 : 0);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + cc * 32, *reinterpret_cast<float(*)[32]>(&x[cc * 32]));
+      tmem_wait_ld();
+      const bool need_mask = !live || (kb + kTileKeys > P) || (kb + kTileKeys > hi);
+      float tmax = -INFINITY;
+      if (!need_mask) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) { x[i] *= p.scale_log2; tmax = fmaxf(tmax, x[i]); }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int j = j0 + i;
+          bool vis = live && j < hi;
+          if (vis && j >= P) {
+            const int nd = j - P;
+            vis = ((nd < 64 ? (mw0 >> nd) : (mw1 >> (nd - 64))) & 1ull) != 0;
+          }
+          x[i] = vis ? x[i] * p.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[i]);
+        }
+      }
+      // combine the two column halves of the row
+      c.xmax[t & 1][h][m] = tmax;
+      named_sync(1, 128);
+      tmax = fmaxf(tmax, c.xmax[t & 1][h ^ 1][m]);
+
+      bool rescale = false;
+      float alpha = 1.f;
+      if (tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax != -INFINITY)) {
+        if (m_used != -INFINITY) {
+          alpha = exp2f(m_used - tmax);
+          rescale = true;
+        }
+        m_used = tmax;
+      }
+      uint32_t pk[64];
+      float sum = 0.f;
+      if (m_used == -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) pk[i] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = exp2f(x[2 * i] - m_used);
+          const float p1 = exp2f(x[2 * i + 1] - m_used);
+          sum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+      }
+      l = l * alpha + sum;
+
+      // PV(t-1) must be done before P is overwritten or O rescaled
+      if (t > 0) {
+        mbar_wait(&c.o_done, (t - 1) & 1, abort);
+        tc_fence_after();
+      }
+      if (rescale && t > 0) {
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          float o[32];
+          const uint32_t oa = tmem + lane_base + kTmemO + cc * 32;
+          tmem_ld32(oa, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(oa, o);
+        }
+        tmem_wait_st();
+      }
+      // P -> shared, K-major 128B-swizzled [64 rows x 64 keys] chunks 2h, 2h+1
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {  // 16 groups of 8 keys
+        const int chunk = 2 * h + (g >> 3);
+        const int k16 = g & 7;  // 16-byte unit within the 128-byte row
+        uint8_t* dst = sP + chunk * kChunkBytes + (m >> 3) * 1024 + (m & 7) * 128 +
+                       ((k16 ^ (m & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(p_ready_leader);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ntiles > 0) {
+      mbar_wait(&c.o_done, (ntiles - 1) & 1, abort);
+      tc_fence_after();
+    }
+    c.xsum[h][m] = l;
+    named_sync(1, 128);
+    named_sync(2, 160);
+    const float lsum = l + c.xsum[h ^ 1][m];
+    const bool bad = !req_ok || c.bad_page || *abort;
+    const bool empty = bad || !(lsum > 0.f) || ntiles == 0;
+    const float inv = empty ? 0.f : 1.f / lsum;
+    const float lse = empty ? -INFINITY : (m_used + log2f(lsum)) * kLn2;
+    if (row_in) {
+      const size_t g = (size_t)b * p.R + row;
+      const size_t rows_total = (size_t)p.B * p.R;
+      for (int nc = 0; nc < 2; ++nc) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          if (ntiles > 0) {
+            tmem_ld32(tmem + lane_base + kTmemO + nc * 128 + cc * 32, o);
+            tmem_wait_ld();
+          }
+          const int col = nc * 256 + h * 128 + cc * 32;
+          if (p.S == 1) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g * kDc + col;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 u;
+              u.x = pack_bf16(empty ? 0.f : o[8 * v + 0] * inv, empty ? 0.f : o[8 * v + 1] * inv);
+              u.y = pack_bf16(empty ? 0.f : o[8 * v + 2] * inv, empty ? 0.f : o[8 * v + 3] * inv);
+              u.z = pack_bf16(empty ? 0.f : o[8 * v + 4] * inv, empty ? 0.f : o[8 * v + 5] * inv);
+              u.w = pack_bf16(empty ? 0.f : o[8 * v + 6] * inv, empty ? 0.f : o[8 * v + 7] * inv);
+              reinterpret_cast<uint4*>(dst)[v] = u;
+            }
+          } else {
+            float* dst = p.o_part + ((size_t)split * rows_total + g) * kDc + col;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<float4*>(dst)[v] =
+                  empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                        : make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
+                                      o[4 * v + 3] * inv);
+          }
+        }
+      }
+      if (h == 0) {
+        if (p.S == 1) p.lse[g] = lse;
+        else p.lse_part[(size_t)split * rows_total + g] = lse;
+      }
+    }
+    if (threadIdx.x == 64 && p.req_status && (!req_ok || c.bad_page))
+      p.req_status[b] = VA_ERR_INVALID_ARG;
+    if (threadIdx.x == 64 && p.req_status && *abort) p.req_status[b] = VA_ERR_CUDA;
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] tensor with [64 x 64] boxes and
+// 128-byte swizzle (the layout the UMMA descriptors above expect).
+bool encode_2d(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = get_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
+                           cudaStream_t st) {
+  if (a.B == 0) return cudaSuccess;
+  const long long R = (long long)a.T * a.H;
+  const long long rows_total = (long long)a.B * R;
+  if (rows_total > 0x7fffffffLL) return cudaErrorNotSupported;
+  CUtensorMap tqn, tqp, tckv, tkpe;
+  if (!encode_2d(&tqn, a.q_nope, rows_total, kDc) || !encode_2d(&tqp, a.q_pe, rows_total, kDr) ||
+      !encode_2d(&tckv, a.c_kv, (uint64_t)a.num_pages * kPage, kDc) ||
+      !encode_2d(&tkpe, a.k_pe, (uint64_t)a.num_pages * kPage, kDr))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  TcParams p;
+  p.page_table = a.page_table;
+  p.kv_len = a.kv_len;
+  p.tree_mask = a.tree_mask;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.req_status = a.req_status;
+  p.B = a.B;
+  p.H = a.H;
+  p.T = a.T;
+  p.R = (int)R;
+  p.max_pages = a.max_pages;
+  p.num_pages = a.num_pages;
+  p.S = S;
+  p.scale_log2 = a.scale * kLog2e;
+  dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)S);
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, p);
+  return cudaGetLastError();
+}
+
 }  // namespace va
+
+extern "C" unsigned int va_device_timeouts(void) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, va::g_tc_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  return v;
+}
