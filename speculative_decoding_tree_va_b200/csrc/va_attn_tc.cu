@@ -441,6 +441,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       const int j0 = kb + 128 * h;  // key of this thread's first column
       mbar_wait(&c.s_full[t & 1], (t >> 1) & 1, abort);
       tc_fence_after();
+      __syncwarp();  // tcgen05.ld is warp-collective
       float x[128];
       const uint32_t s_addr = tmem + lane_base + ((t & 1) ? kTmemS1 : 0);
 #pragma unroll
@@ -499,7 +500,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         mbar_wait(&c.o_done, (t - 1) & 1, abort);
         tc_fence_after();
       }
-      if (rescale && t > 0) {
+      // tcgen05.ld/st are warp-collective: the whole warp takes this branch
+      // if any of its rows needs it (factor 1 for the others)
+      __syncwarp();
+      if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+        const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
           float o[32];
@@ -507,7 +512,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           tmem_ld32(oa, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          for (int i = 0; i < 32; ++i) o[i] *= f;
           tmem_st32(oa, o);
         }
         tmem_wait_st();
@@ -540,8 +545,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     const bool empty = bad || !(lsum > 0.f) || ntiles == 0;
     const float inv = empty ? 0.f : 1.f / lsum;
     const float lse = empty ? -INFINITY : (m_used + log2f(lsum)) * kLn2;
-    if (row_in) {
-      const size_t g = (size_t)b * p.R + row;
+    __syncwarp();
+    {
+      // every lane runs the (warp-collective) TMEM loads; only rows inside
+      // the request store
+      const size_t g = (size_t)b * p.R + (row_in ? row : 0);
       const size_t rows_total = (size_t)p.B * p.R;
       for (int nc = 0; nc < 2; ++nc) {
 #pragma unroll 1
@@ -552,7 +560,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
             tmem_wait_ld();
           }
           const int col = nc * 256 + h * 128 + cc * 32;
-          if (p.S == 1) {
+          if (!row_in) {
+            // nothing to store for rows past the request
+          } else if (p.S == 1) {
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g * kDc + col;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -572,9 +582,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
                         : make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
                                       o[4 * v + 3] * inv);
           }
+          __syncwarp();  // reconverge before the next warp-collective load
         }
       }
-      if (h == 0) {
+      if (h == 0 && row_in) {
         if (p.S == 1) p.lse[g] = lse;
         else p.lse_part[(size_t)split * rows_total + g] = lse;
       }
@@ -585,6 +596,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   }
 
   // ------------------------------------------------------------------ teardown
+  __syncwarp();  // role branches diverge inside warps 0 and 1; reconverge first
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();

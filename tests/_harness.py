@@ -56,8 +56,17 @@ def compare(out_gpu, lse_gpu, out_ref, lse_ref, dtype: str, what: str = ""):
     assert np.array_equal(np.isneginf(lse_gpu), empty), f"{what}: empty-row pattern differs"
     assert not out_gpu[empty].any(), f"{what}: absent rows not zero"
     assert np.isfinite(out_gpu).all() and np.isfinite(lse_gpu[~empty]).all(), f"{what}: non-finite"
-    d_out = float(np.abs(out_gpu - out_ref).max()) if out_ref.size else 0.0
+    err = np.abs(out_gpu - out_ref)
+    d_out = float(err.max()) if out_ref.size else 0.0
     d_lse = float(np.abs(lse_gpu[~empty] - lse_ref[~empty]).max()) if (~empty).any() else 0.0
-    assert d_out <= tol["out"], f"{what}: out max_abs {d_out:.3e} > {tol['out']}"
+    if dtype == "bf16":
+        # bf16 outputs: the bar is 1e-2, except where storing the exact value
+        # in bf16 alone costs more (half an ulp = 2^-8 |x| reaches 1e-2 at
+        # |x| >= 2.56); there the storage rounding plus 2e-3 is allowed.
+        bar = np.maximum(tol["out"], np.abs(out_ref) * 2.0 ** -8 + 2e-3)
+        worst = float((err - bar).max()) if out_ref.size else -1.0
+        assert worst <= 0, f"{what}: out max_abs {d_out:.3e} over the bf16 bar"
+    else:
+        assert d_out <= tol["out"], f"{what}: out max_abs {d_out:.3e} > {tol['out']}"
     assert d_lse <= tol["lse"], f"{what}: lse max_abs {d_lse:.3e} > {tol['lse']}"
     return d_out, d_lse
