@@ -1,0 +1,379 @@
+"""Throughput of the DDTree tree-verify step (mask + MLA-absorb attention) on B200.
+
+One step = va_build_tree_mask + va_verify_attn (+ va_merge when split) over one
+batch of synthetic requests, inputs resident in HBM.  Default workload:
+bf16, B = 64 requests, H = 64 heads, prefix P ~ U[512, 8192] per request,
+tree budget 32 (T = 33) best-first trees, 64-token shuffled pages.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is TFLOP/s of algorithmic work
+(visible keys only) over the whole job; `e2e` is the same metric through the
+public binding with host buffers (pinned host -> device copies of the
+step's queries and tree, result copied back, inside the timed region; the
+KV cache stays resident).  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_decoding_tree_va_b200 import synth  # noqa: E402
+
+METRIC = ("verify-attn TFLOP/s & % of B200 roofline; µs per tree-verify step at B=64")
+FLOP_PER_KEY = 2 * (synth.D_LATENT + synth.D_ROPE) + 2 * synth.D_LATENT  # QK + PV per (row, key)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return m["hbm_gbs"], m["bf16_tflops"], m.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def work(inp, depth):
+    """Algorithmic flops and bytes of one step (visible keys only)."""
+    B, T, H = inp.wl.B, inp.T, inp.wl.H
+    e = 2 if inp.wl.dtype == "bf16" else 4
+    present = depth >= 0                                    # [B, T]
+    vis = (inp.prefix[:, None].astype(np.int64) + depth + 1) * present
+    flops = float(vis.sum()) * H * FLOP_PER_KEY
+    kv_bytes = float(inp.kv_len.astype(np.int64).sum()) * (synth.D_LATENT + synth.D_ROPE) * e
+    q_bytes = float(B * T * H) * (synth.D_LATENT + synth.D_ROPE) * e
+    out_bytes = float(B * T * H) * (synth.D_LATENT * e + 4)
+    return flops, kv_bytes + q_bytes + out_bytes
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                mx = float(f[2].split()[0])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * (mx or 1)] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    if n_gpus > 1:
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return rank, local, dist
+    torch.cuda.set_device(0)
+    return 0, 0, None
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(args):
+    import torch
+    import speculative_decoding_tree_va_b200 as va
+
+    rank, local, dist = dist_setup(args.gpus)
+    wl = synth.WORKLOADS[args.workload]
+    # every rank verifies its own batch (independent requests): weak scaling
+    inp = synth.make_inputs(wl, seed=wl.seed + 7919 * rank)
+    dev = torch.device("cuda", local)
+    bf16 = wl.dtype == "bf16"
+    tdt = torch.bfloat16 if bf16 else torch.float32
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if bf16:
+            t = t.view(torch.int16).view(torch.bfloat16)
+        return t.to(dev)
+
+    q_nope, q_pe = to_dev(inp.q_nope), to_dev(inp.q_pe)
+    c_kv, k_pe = to_dev(inp.c_kv), to_dev(inp.k_pe)
+    page_table = torch.from_numpy(inp.page_table).to(dev)
+    kv_len = torch.from_numpy(inp.kv_len).to(dev)
+    # draft trees from the library's GPU best-first builder
+    parents, _, depth, _ = va.build_tree(torch.from_numpy(inp.lp).to(dev),
+                                         torch.from_numpy(inp.tok).to(dev), wl.budget)
+    depth_h = depth.cpu().numpy()
+    flops, alg_bytes = work(inp, depth_h)
+    B, T, H = wl.B, wl.T, wl.H
+    out = torch.empty(B, T, H, synth.D_LATENT, device=dev, dtype=tdt)
+    lse = torch.empty(B, T, H, device=dev, dtype=torch.float32)
+    mask = torch.empty(B, T, (T + 63) // 64, device=dev, dtype=torch.int64)
+    tstat = torch.empty(B, device=dev, dtype=torch.int32)
+    splits = args.splits if args.splits is not None else wl.splits
+    vargs = va.make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, out, lse,
+                         scale=synth.SCALE, num_splits=splits)
+    S = va.num_splits(vargs)
+    wbytes = va.workspace_bytes(vargs)
+    ws = torch.empty(max(wbytes, 256), device=dev, dtype=torch.uint8) if wbytes else None
+    if ws is not None:
+        vargs.workspace, vargs.workspace_bytes = ws.data_ptr(), wbytes
+    lib = va.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sptr = va._stream(stream)
+    import ctypes
+
+    def step(ev_a=None, ev_b=None):
+        r = lib.va_build_tree_mask(ctypes.c_void_p(parents.data_ptr()), B, T,
+                                   ctypes.c_void_p(mask.data_ptr()),
+                                   ctypes.c_void_p(tstat.data_ptr()), sptr)
+        if ev_a is not None:
+            ev_a.record(stream)
+        r |= lib.va_verify_attn(ctypes.byref(vargs), sptr)
+        if ev_b is not None:
+            ev_b.record(stream)
+        if r:
+            raise RuntimeError("library call failed")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # timed region: K back-to-back steps, inputs (> 126 MB L2) resident in HBM
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for a, b in evs:
+            step(a, b)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(ms_total, dist)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ms_step = ms_total / args.steps
+    world = args.gpus
+    value = flops * world / (ms_step * 1e-3) / 1e12
+
+    # end to end through the binding with host buffers
+    def host(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if bf16 else a).pin_memory()
+
+    q_nope_h, q_pe_h = host(inp.q_nope), host(inp.q_pe)
+    par_h = parents.cpu().pin_memory()
+    kv_h = torch.from_numpy(inp.kv_len).pin_memory()
+    pt_h = torch.from_numpy(inp.page_table).pin_memory()
+    out_h = torch.empty(out.numel() * out.element_size(), dtype=torch.uint8).pin_memory()
+    lse_h = torch.empty(lse.numel(), dtype=torch.float32).pin_memory()
+    qn_d = q_nope.view(torch.int16) if bf16 else q_nope
+    qp_d = q_pe.view(torch.int16) if bf16 else q_pe
+    h2d = sum(x.numel() * x.element_size() for x in (q_nope_h, q_pe_h, par_h, kv_h, pt_h))
+    d2h = out.numel() * out.element_size() + lse.numel() * 4
+
+    def e2e_step():
+        qn_d.copy_(q_nope_h, non_blocking=True)
+        qp_d.copy_(q_pe_h, non_blocking=True)
+        parents.copy_(par_h, non_blocking=True)
+        kv_len.copy_(kv_h, non_blocking=True)
+        page_table.copy_(pt_h, non_blocking=True)
+        step()
+        out_h.copy_(out.view(-1).view(torch.uint8), non_blocking=True)
+        lse_h.copy_(lse.view(-1), non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist)
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    hbm, tc_peak, tc_sust, peak_src = peaks()
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roof_us = max(flops / (tc_peak * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
+    clocks = clk.summary()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None if args.no_cpu_baseline else cpu_baseline(inp, depth_h, budget_s=args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "us_per_step": round(ms_step * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded; no dataset or weights)",
+        "config": {"workload": wl.name, "B": B, "H": H, "T": T,
+                   "prefix": list(wl.P) if isinstance(wl.P, tuple) else wl.P,
+                   "tree": f"best-first top-{wl.topk}, depth<={wl.max_depth}, budget {wl.budget}",
+                   "kv": "64-token pages, shuffled" if wl.paged else "contiguous",
+                   "num_splits": S, "parallelism": f"replicas x{world} (independent requests)",
+                   "l2": "inputs larger than the 126 MB L2, no flush",
+                   "gflop_per_step": round(flops / 1e9, 2), "alg_mb_per_step": round(alg_bytes / 1e6, 1)},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst); sustained {tc_sust}",
+                     "kernel": "attn_tc_kernel" if bf16 else "attn_simt_kernel",
+                     "kernel_us": round(attn_ms * 1e3, 1), "roofline_us": round(roof_us, 1),
+                     "frac_of_step_roofline": round(roof_us / (ms_step * 1e3), 4)},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": args.steps * (2 + (1 if S > 1 else 0)),
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(inp, depth, budget_s=15.0):
+    """fp64 oracle, single-threaded, on a seeded sample of whole rows."""
+    import oracle
+    B, T, H = inp.wl.B, inp.T, inp.wl.H
+    trees = oracle.build_trees(inp.lp, inp.tok, inp.wl.budget)
+    mask, _ = oracle.ancestor_mask(trees["parent"])
+    rng = np.random.default_rng(12345)
+    order = rng.permutation(B * T * H).astype(np.int32)
+    done_rows, flops, t_used = 0, 0.0, 0.0
+    chunk = 32
+    while t_used < budget_s and done_rows < order.size:
+        rows = order[done_rows:done_rows + chunk]
+        t0 = time.perf_counter()
+        oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe, inp.page_table,
+                              inp.kv_len, mask, scale=synth.SCALE, dtype=inp.wl.dtype, rows=rows)
+        t_used += time.perf_counter() - t0
+        b = rows // (T * H)
+        t = (rows // H) % T
+        d = trees["depth"][b, t]
+        flops += float(((inp.prefix[b].astype(np.int64) + d + 1) * (d >= 0)).sum()) * FLOP_PER_KEY
+        done_rows += rows.size
+    return {"value": round(flops / t_used / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{done_rows} seeded (b,t,h) rows of {B * T * H}, {t_used:.1f} s, fp64 C++"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: fp64 C++ on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl)
+    import oracle
+    trees = oracle.build_trees(inp.lp, inp.tok, wl.budget)
+    depth = trees["depth"]
+    per_step = max(2.0, args.cpu_seconds / max(args.steps, 1))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, depth, budget_s=0.2)
+    vals = [cpu_baseline(inp, depth, budget_s=per_step) for _ in range(args.steps)]
+    v = float(np.mean([x["value"] for x in vals]))
+    flops, _ = work(inp, depth)
+    ms = flops / (v * 1e12) * 1e3
+    line = {
+        "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; no dataset or weights)", "impl": "reference",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T,
+                   "note": "each step = a bounded row sample; per-step time extrapolated per flop"},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": vals[0]["sample"]},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="bf16-b64-ragged", choices=list(synth.WORKLOADS))
+    ap.add_argument("--splits", type=int, default=None)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
