@@ -43,7 +43,11 @@ __device__ unsigned int g_tc_timeouts = 0;  // count of barrier waits that expir
 
 namespace {
 
-constexpr int kThreads = 192;          // 6 warps
+constexpr int kThreads = 256;          // 8 warps
+constexpr int kLoadWarps = 2;          // warps 6-7: cp.async loaders
+constexpr int kLoadThreads = 32 * kLoadWarps;
+constexpr int kTmaK = 9;               // K chunks 0..kTmaK-1 of a tile come by TMA, the rest by cp.async
+constexpr int kCpDepth = 3;            // slots of cp.async groups in flight per loader thread
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
 constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
@@ -55,6 +59,8 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr unsigned long long kTimeoutNs = 1000000000ull;
 
 struct TcParams {
+  const void* c_kv;
+  const void* k_pe;
   const int32_t* page_table;
   const int32_t* kv_len;
   const uint64_t* tree_mask;
@@ -68,7 +74,8 @@ struct TcParams {
 };
 
 struct __align__(16) Ctl {
-  uint64_t full[kRing];
+  uint64_t full[kRing];   // TMA-filled slots: leader's expect_tx + bytes from both CTAs
+  uint64_t fullL[kRing];  // cp.async-filled slots: one arrival per loader warp of both CTAs
   uint64_t empty[kRing];
   uint64_t q_full;
   uint64_t s_full[2];
@@ -260,7 +267,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   const int ntiles = hi > lo ? (hi - lo + kTileKeys - 1) / kTileKeys : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRing; ++s) { mbar_init(&c.full[s], 1); mbar_init(&c.empty[s], 1); }
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.fullL[s], 2 * kLoadWarps);
+      mbar_init(&c.empty[s], 1);
+    }
     mbar_init(&c.q_full, 1);
     mbar_init(&c.s_full[0], 1);
     mbar_init(&c.s_full[1], 1);
@@ -313,28 +324,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         const int r0 = page_row(kb / kPage + 2 * (int)rank);
         const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
         for (int kc = 0; kc < 9; ++kc) {
-          const uint32_t bar = acquire();
-          const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-          const CUtensorMap* m = kc < 8 ? &tm_ckv : &tm_kpe;
-          const int x = kc < 8 ? kc * 64 : 0;
-          tma_load_2d(dst, m, bar, x, r0);
-          tma_load_2d(dst + kChunkBytes, m, bar, x, r1);
+          if (kc < kTmaK) {
+            const uint32_t bar = acquire();
+            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+            const CUtensorMap* m = kc < 8 ? &tm_ckv : &tm_kpe;
+            const int x = kc < 8 ? kc * 64 : 0;
+            tma_load_2d(dst, m, bar, x, r0);
+            tma_load_2d(dst + kChunkBytes, m, bar, x, r1);
+          }
           advance();
         }
       };
-      auto load_v = [&](int t) {
+      auto load_v = [&](int t) {  // V slots come from the cp.async loaders
         const int kb = lo + t * kTileKeys;
         for (int pg = 0; pg < 4; ++pg) {
           if (kb + pg * kPage >= hi) break;
-          const int r = page_row(kb / kPage + pg);
-          for (int nc = 0; nc < 2; ++nc) {
-            const uint32_t bar = acquire();
-            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-            const int x = nc * 256 + (int)rank * 128;
-            tma_load_2d(dst, &tm_ckv, bar, x, r);
-            tma_load_2d(dst + kChunkBytes, &tm_ckv, bar, x + 64, r);
-            advance();
-          }
+          advance();
+          advance();
         }
       };
       for (int t = 0; t < ntiles; ++t) {
@@ -370,7 +376,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       auto qk = [&](int t) {
         const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
         for (int kc = 0; kc < 9; ++kc) {
-          mbar_wait(&c.full[slot], phase, abort);
+          mbar_wait(kc < kTmaK ? &c.full[slot] : &c.fullL[slot], phase, abort);
           tc_fence_after();
           const uint32_t kslot = sr + slot * kSlotBytes;
 #pragma unroll
@@ -391,7 +397,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         for (int pg = 0; pg < 4; ++pg) {
           if (kb + pg * kPage >= hi) break;
           for (int nc = 0; nc < 2; ++nc) {
-            mbar_wait(&c.full[slot], phase, abort);
+            mbar_wait(&c.fullL[slot], phase, abort);
             tc_fence_after();
             const uint32_t vslot = sr + slot * kSlotBytes;
             const uint32_t d = tmem + kTmemO + nc * 128;
@@ -414,6 +420,114 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         if (t > 0) pv(t - 1);
       }
       pv(ntiles - 1);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ cp.async loaders
+    // Thread-issued 16-byte copies run beside the TMA engine (whose per-SM
+    // throughput alone cannot feed the tensor cores here).  Keys at or past
+    // the split end are zero-filled, so V rows the softmax masks out are exact
+    // zeros whatever the page holds.
+    if (ntiles > 0) {
+      const int tl = threadIdx.x - 6 * 32;  // 0..63
+      const int npages_valid = (kv_len + kPage - 1) / kPage;
+      const __nv_bfloat16* ckv = reinterpret_cast<const __nv_bfloat16*>(p.c_kv);
+      const __nv_bfloat16* kpe = reinterpret_cast<const __nv_bfloat16*>(p.k_pe);
+      auto phys_of = [&](int pg) -> int {
+        if (pg >= npages_valid) return -1;
+        const int ph = p.page_table[(size_t)b * p.max_pages + pg];
+        return (ph < 0 || ph >= p.num_pages) ? -1 : ph;
+      };
+      int slot = 0, pos = 0, last_pos = -2;
+      uint32_t phase = 0;
+      int pend_slot[kCpDepth];
+      int npend = 0, head = 0;
+      auto advance = [&]() { ++pos; if (++slot == kRing) { slot = 0; phase ^= 1; } };
+      auto signal_oldest = [&]() {
+        const int s = pend_slot[head];
+        head = (head + 1 == kCpDepth) ? 0 : head + 1;
+        --npend;
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&c.fullL[s]), 0));
+      };
+      auto begin_slot = [&]() {
+        // A slot still unsignalled must never wait behind a ring position
+        // that only its own consumption can free: flush before any gap.
+        if (npend > 0 && pos != last_pos + 1) {
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
+          while (npend > 0) signal_oldest();
+        }
+        last_pos = pos;
+        if (lane == 0) mbar_wait(&c.empty[slot], phase ^ 1, abort);
+        __syncwarp();
+      };
+      auto end_slot = [&]() {
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        int tail = head + npend;
+        if (tail >= kCpDepth) tail -= kCpDepth;
+        pend_slot[tail] = slot;
+        ++npend;
+        if (npend == kCpDepth) {
+          asm volatile("cp.async.wait_group %0;" ::"n"(kCpDepth - 1) : "memory");
+          signal_oldest();
+        }
+        advance();
+      };
+      auto cp16 = [&](uint32_t dst, const void* src, bool valid) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                     ::"r"(dst), "l"(valid ? src : p.c_kv), "r"(valid ? 16 : 0) : "memory");
+      };
+      for (int t = 0; t <= ntiles; ++t) {
+        if (t < ntiles) {  // K chunks kTmaK..8 of tile t
+          const int kb = lo + t * kTileKeys;
+          const int ph0 = phys_of(kb / kPage + 2 * (int)rank);
+          const int ph1 = phys_of(kb / kPage + 2 * (int)rank + 1);
+          for (int kc = 0; kc < 9; ++kc) {
+            if (kc < kTmaK) { advance(); continue; }
+            begin_slot();
+            const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+              const int cidx = tl + kLoadThreads * k;  // 1024 16-byte units
+              const int r = cidx >> 3, u = cidx & 7;   // r: key 0..127 of this CTA
+              const int ph = (r >> 6) ? ph1 : ph0;
+              const size_t krow = (size_t)(ph < 0 ? 0 : ph) * kPage + (r & 63);
+              const void* src = kc < 8 ? (const void*)(ckv + krow * kDc + kc * 64 + u * 8)
+                                       : (const void*)(kpe + krow * kDr + u * 8);
+              const uint32_t dst = sbase + (r >> 6) * kChunkBytes + (r & 63) * 128 + ((u ^ (r & 7)) << 4);
+              cp16(dst, src, ph >= 0);
+            }
+            end_slot();
+          }
+        }
+        if (t > 0) {  // V slots of tile t-1: [64 keys x 128 latent columns] per page and chunk
+          const int kb = lo + (t - 1) * kTileKeys;
+          for (int pg = 0; pg < 4; ++pg) {
+            const int k0 = kb + pg * kPage;
+            if (k0 >= hi) break;
+            const int ph = phys_of(k0 / kPage);
+            for (int nc = 0; nc < 2; ++nc) {
+              begin_slot();
+              const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
+              const int col0 = nc * 256 + (int)rank * 128;
+#pragma unroll 4
+              for (int k = 0; k < 16; ++k) {
+                const int cidx = tl + kLoadThreads * k;
+                const int r = cidx >> 4, u16 = cidx & 15;  // r: key in page, u16: 16 B unit of 256 B
+                const int sub = u16 >> 3, u = u16 & 7;
+                const bool valid = ph >= 0 && k0 + r < hi;
+                const size_t krow = (size_t)(ph < 0 ? 0 : ph) * kPage + r;
+                const void* src = ckv + krow * kDc + col0 + u16 * 8;
+                const uint32_t dst = sbase + sub * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4);
+                cp16(dst, src, valid);
+              }
+              end_slot();
+            }
+          }
+        }
+      }
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      while (npend > 0) signal_oldest();
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -652,6 +766,8 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   TcParams p;
+  p.c_kv = a.c_kv;
+  p.k_pe = a.k_pe;
   p.page_table = a.page_table;
   p.kv_len = a.kv_len;
   p.tree_mask = a.tree_mask;
