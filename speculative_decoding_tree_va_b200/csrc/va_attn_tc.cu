@@ -81,6 +81,7 @@ struct __align__(16) Ctl {
   uint64_t s_full[2];
   uint64_t p_ready;
   uint64_t o_done;
+  uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
   int bad_page;
@@ -142,6 +143,18 @@ __device__ __noinline__ bool mbar_wait(uint64_t* barp, uint32_t parity, volatile
       return false;
     }
   }
+}
+// Last-resort wait used only after an abort (bounded, never marks anything).
+__device__ __noinline__ void mbar_wait_final(uint64_t* barp, uint32_t parity) {
+  const uint32_t bar = smem_u32(barp);
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try(bar, parity))
+    if (global_ns() - t0 > kTimeoutNs) return;
+}
+// After an abort: give copies already in flight time to land (bounded).
+__device__ __noinline__ void settle() {
+  const unsigned long long t0 = global_ns();
+  while (global_ns() - t0 < 200000ull) { }
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar_cluster, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
@@ -277,6 +290,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     mbar_init(&c.s_full[1], 1);
     mbar_init(&c.p_ready, 8);  // 4 softmax warps x 2 CTAs
     mbar_init(&c.o_done, 1);
+    mbar_init(&c.mma_drain, 1);
     c.abort = 0;
     c.bad_page = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -313,7 +327,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       int slot = 0;
       uint32_t phase = 0;
       auto acquire = [&]() -> uint32_t {  // wait for a free slot, post the byte count
-        mbar_wait(&c.empty[slot], phase ^ 1, abort);
+        if (!mbar_wait(&c.empty[slot], phase ^ 1, abort)) return 0u;
         const uint32_t bar = map_to_rank(smem_u32(&c.full[slot]), 0);
         if (rank == 0) mbar_arrive_expect_tx(bar, 2 * kSlotBytes);
         return bar;
@@ -324,8 +338,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         const int r0 = page_row(kb / kPage + 2 * (int)rank);
         const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
         for (int kc = 0; kc < 9; ++kc) {
+          if (*abort) return;
           if (kc < kTmaK) {
             const uint32_t bar = acquire();
+            if (!bar) return;
             const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
             const CUtensorMap* m = kc < 8 ? &tm_ckv : &tm_kpe;
             const int x = kc < 8 ? kc * 64 : 0;
@@ -343,16 +359,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           advance();
         }
       };
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = 0; t < ntiles && !*abort; ++t) {
         load_k(t);
         if (t > 0) load_v(t - 1);
       }
-      load_v(ntiles - 1);
+      if (!*abort) load_v(ntiles - 1);
       // drain: every slot's last load must be consumed before the CTA may exit
-      for (int s = 0; s < kRing; ++s) {
+      for (int s = 0; s < kRing && !*abort; ++s) {
         mbar_wait(&c.empty[slot], phase ^ 1, abort);
         advance();
       }
+      if (*abort) settle();  // loads already issued land before teardown
     } else if (lane > 0 && ntiles > 0) {
       // the other 31 lanes check every page index this split reads
       int bad = 0;
@@ -370,13 +387,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
       const uint32_t sq = smem_u32(sQ), sp = smem_u32(sP), sr = smem_u32(sRing);
       int slot = 0;
-      uint32_t phase = 0;
-      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      mbar_wait(&c.q_full, 0, abort);
+      // Each slot's two full barriers complete once per use of their own
+      // kind, so each keeps its own phase bit per slot.
+      uint32_t bitsT = 0, bitsL = 0;
+      auto advance = [&]() { if (++slot == kRing) slot = 0; };
+      auto wait_full = [&](bool tma) -> bool {
+        uint32_t& bits = tma ? bitsT : bitsL;
+        const bool ok = mbar_wait(tma ? &c.full[slot] : &c.fullL[slot], (bits >> slot) & 1u, abort);
+        bits ^= 1u << slot;
+        return ok;
+      };
+      bool ok = mbar_wait(&c.q_full, 0, abort);
       auto qk = [&](int t) {
         const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
-        for (int kc = 0; kc < 9; ++kc) {
-          mbar_wait(kc < kTmaK ? &c.full[slot] : &c.fullL[slot], phase, abort);
+        for (int kc = 0; kc < 9 && ok; ++kc) {
+          ok = wait_full(kc < kTmaK);
+          if (!ok) break;
           tc_fence_after();
           const uint32_t kslot = sr + slot * kSlotBytes;
 #pragma unroll
@@ -392,12 +418,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       };
       auto pv = [&](int t) {
         const int kb = lo + t * kTileKeys;
-        mbar_wait(&c.p_ready, t & 1, abort);
+        if (ok) ok = mbar_wait(&c.p_ready, t & 1, abort);
+        if (!ok) return;
         tc_fence_after();
-        for (int pg = 0; pg < 4; ++pg) {
+        for (int pg = 0; pg < 4 && ok; ++pg) {
           if (kb + pg * kPage >= hi) break;
-          for (int nc = 0; nc < 2; ++nc) {
-            mbar_wait(&c.fullL[slot], phase, abort);
+          for (int nc = 0; nc < 2 && ok; ++nc) {
+            ok = wait_full(false);
+            if (!ok) break;
             tc_fence_after();
             const uint32_t vslot = sr + slot * kSlotBytes;
             const uint32_t d = tmem + kTmemO + nc * 128;
@@ -415,11 +443,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         }
         mma_commit_pair(&c.o_done);
       };
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = 0; t < ntiles && ok; ++t) {
         qk(t);
         if (t > 0) pv(t - 1);
       }
-      pv(ntiles - 1);
+      if (ok) pv(ntiles - 1);
+      if (!ok) {
+        // aborted: issue nothing more, and let every MMA already issued
+        // finish before the pair tears down and frees tensor memory
+        mma_commit_pair(&c.mma_drain);
+        mbar_wait_final(&c.mma_drain, 0);
+      }
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ cp.async loaders
@@ -460,6 +494,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         last_pos = pos;
         if (lane == 0) mbar_wait(&c.empty[slot], phase ^ 1, abort);
         __syncwarp();
+        return !*abort;
       };
       auto end_slot = [&]() {
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -477,14 +512,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                      ::"r"(dst), "l"(valid ? src : p.c_kv), "r"(valid ? 16 : 0) : "memory");
       };
-      for (int t = 0; t <= ntiles; ++t) {
+      for (int t = 0; t <= ntiles && !*abort; ++t) {
         if (t < ntiles) {  // K chunks kTmaK..8 of tile t
           const int kb = lo + t * kTileKeys;
           const int ph0 = phys_of(kb / kPage + 2 * (int)rank);
           const int ph1 = phys_of(kb / kPage + 2 * (int)rank + 1);
           for (int kc = 0; kc < 9; ++kc) {
             if (kc < kTmaK) { advance(); continue; }
-            begin_slot();
+            if (!begin_slot()) break;
             const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
 #pragma unroll 4
             for (int k = 0; k < 16; ++k) {
@@ -507,7 +542,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
             if (k0 >= hi) break;
             const int ph = phys_of(k0 / kPage);
             for (int nc = 0; nc < 2; ++nc) {
-              begin_slot();
+              if (!begin_slot()) break;
               const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
               const int col0 = nc * 256 + (int)rank * 128;
 #pragma unroll 4
