@@ -46,7 +46,6 @@ namespace {
 constexpr int kThreads = 256;          // 8 warps
 constexpr int kLoadWarps = 2;          // warps 6-7: cp.async loaders
 constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kTmaK = 9;               // K chunks 0..kTmaK-1 of a tile come by TMA, the rest by cp.async
 constexpr int kCpDepth = 3;            // slots of cp.async groups in flight per loader thread
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
@@ -74,8 +73,7 @@ struct TcParams {
 };
 
 struct __align__(16) Ctl {
-  uint64_t full[kRing];   // TMA-filled slots: leader's expect_tx + bytes from both CTAs
-  uint64_t fullL[kRing];  // cp.async-filled slots: one arrival per loader warp of both CTAs
+  uint64_t full[kRing];   // leader's expect_tx arrival + TMA bytes + loader-warp arrivals
   uint64_t empty[kRing];
   uint64_t q_full;
   uint64_t s_full[2];
@@ -281,8 +279,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&c.full[s], 1);
-      mbar_init(&c.fullL[s], 2 * kLoadWarps);
+      mbar_init(&c.full[s], 1 + 2 * kLoadWarps);
       mbar_init(&c.empty[s], 1);
     }
     mbar_init(&c.q_full, 1);
@@ -306,8 +303,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   const uint32_t tmem = c.tmem_base;
   volatile int* abort = &c.abort;
 
+  // Ring protocol.  Every 16 KB slot is two 8 KB boxes: box A comes by TMA,
+  // box B by the cp.async loader warps, so both copy engines of the SM work on
+  // every slot.  Each producer and the MMA issuer walk the same slot sequence
+  // -- for tile t: K chunks kc = 0..8 of tile t, then the V slots of tile t-1 --
+  // so every ring position is taken by each of them in order and a barrier
+  // phase can never be waited on twice ahead.  A slot is full when the
+  // leader's expect_tx arrival, both CTAs' TMA bytes and one arrival per
+  // loader warp of both CTAs are in.  V slots of a page that ends inside the
+  // key range (or is invalid) are loaded entirely by the loaders, which
+  // zero-fill keys past the range, so the TMA side posts no bytes for them.
+  auto v_partial = [&](int k0) -> bool { return k0 + kPage > hi; };
+
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0 && ntiles > 0) {
       const uint32_t q_bar = map_to_rank(smem_u32(&c.q_full), 0);
       if (rank == 0) mbar_arrive_expect_tx(q_bar, 2 * kQBytes);
@@ -326,47 +335,50 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       };
       int slot = 0;
       uint32_t phase = 0;
-      auto acquire = [&]() -> uint32_t {  // wait for a free slot, post the byte count
-        if (!mbar_wait(&c.empty[slot], phase ^ 1, abort)) return 0u;
-        const uint32_t bar = map_to_rank(smem_u32(&c.full[slot]), 0);
-        if (rank == 0) mbar_arrive_expect_tx(bar, 2 * kSlotBytes);
-        return bar;
-      };
       auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      auto load_k = [&](int t) {
-        const int kb = lo + t * kTileKeys;
-        const int r0 = page_row(kb / kPage + 2 * (int)rank);
-        const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
-        for (int kc = 0; kc < 9; ++kc) {
-          if (*abort) return;
-          if (kc < kTmaK) {
-            const uint32_t bar = acquire();
-            if (!bar) return;
-            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-            const CUtensorMap* m = kc < 8 ? &tm_ckv : &tm_kpe;
-            const int x = kc < 8 ? kc * 64 : 0;
-            tma_load_2d(dst, m, bar, x, r0);
-            tma_load_2d(dst + kChunkBytes, m, bar, x, r1);
+      // wait for the slot, post this slot's TMA bytes; false on abort
+      auto acquire = [&](uint32_t bytes, uint32_t* bar) -> bool {
+        if (!mbar_wait(&c.empty[slot], phase ^ 1, abort)) return false;
+        *bar = map_to_rank(smem_u32(&c.full[slot]), 0);
+        if (rank == 0) mbar_arrive_expect_tx(*bar, 2 * bytes);
+        return true;
+      };
+      bool go = true;
+      for (int t = 0; t <= ntiles && go; ++t) {
+        if (t < ntiles) {  // K chunks: box A = this CTA's first page of the tile
+          const int kb = lo + t * kTileKeys;
+          const int r0 = page_row(kb / kPage + 2 * (int)rank);
+          for (int kc = 0; kc < 9 && go; ++kc) {
+            uint32_t bar;
+            go = acquire(kChunkBytes, &bar);
+            if (!go) break;
+            tma_load_2d(smem_u32(sRing + (size_t)slot * kSlotBytes), kc < 8 ? &tm_ckv : &tm_kpe,
+                        bar, kc < 8 ? kc * 64 : 0, r0);
+            advance();
           }
-          advance();
         }
-      };
-      auto load_v = [&](int t) {  // V slots come from the cp.async loaders
-        const int kb = lo + t * kTileKeys;
-        for (int pg = 0; pg < 4; ++pg) {
-          if (kb + pg * kPage >= hi) break;
-          advance();
-          advance();
+        if (t > 0 && go) {  // V slots of tile t-1: box A = the first 64 latent columns
+          const int kb = lo + (t - 1) * kTileKeys;
+          for (int pg = 0; pg < 4 && go; ++pg) {
+            const int k0 = kb + pg * kPage;
+            if (k0 >= hi) break;
+            const bool part = v_partial(k0);
+            const int r = page_row(k0 / kPage);
+            for (int nc = 0; nc < 2 && go; ++nc) {
+              uint32_t bar;
+              go = acquire(part ? 0u : (uint32_t)kChunkBytes, &bar);
+              if (!go) break;
+              if (!part)
+                tma_load_2d(smem_u32(sRing + (size_t)slot * kSlotBytes), &tm_ckv, bar,
+                            nc * 256 + (int)rank * 128, r);
+              advance();
+            }
+          }
         }
-      };
-      for (int t = 0; t < ntiles && !*abort; ++t) {
-        load_k(t);
-        if (t > 0) load_v(t - 1);
       }
-      if (!*abort) load_v(ntiles - 1);
       // drain: every slot's last load must be consumed before the CTA may exit
-      for (int s = 0; s < kRing && !*abort; ++s) {
-        mbar_wait(&c.empty[slot], phase ^ 1, abort);
+      for (int s2 = 0; s2 < kRing && go; ++s2) {
+        go = mbar_wait(&c.empty[slot], phase ^ 1, abort);
         advance();
       }
       if (*abort) settle();  // loads already issued land before teardown
@@ -387,21 +399,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
       const uint32_t sq = smem_u32(sQ), sp = smem_u32(sP), sr = smem_u32(sRing);
       int slot = 0;
-      // Each slot's two full barriers complete once per use of their own
-      // kind, so each keeps its own phase bit per slot.
-      uint32_t bitsT = 0, bitsL = 0;
-      auto advance = [&]() { if (++slot == kRing) slot = 0; };
-      auto wait_full = [&](bool tma) -> bool {
-        uint32_t& bits = tma ? bitsT : bitsL;
-        const bool ok = mbar_wait(tma ? &c.full[slot] : &c.fullL[slot], (bits >> slot) & 1u, abort);
-        bits ^= 1u << slot;
-        return ok;
-      };
+      uint32_t phase = 0;
+      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
       bool ok = mbar_wait(&c.q_full, 0, abort);
       auto qk = [&](int t) {
         const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
         for (int kc = 0; kc < 9 && ok; ++kc) {
-          ok = wait_full(kc < kTmaK);
+          ok = mbar_wait(&c.full[slot], phase, abort);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kslot = sr + slot * kSlotBytes;
@@ -424,7 +428,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         for (int pg = 0; pg < 4 && ok; ++pg) {
           if (kb + pg * kPage >= hi) break;
           for (int nc = 0; nc < 2 && ok; ++nc) {
-            ok = wait_full(false);
+            ok = mbar_wait(&c.full[slot], phase, abort);
             if (!ok) break;
             tc_fence_after();
             const uint32_t vslot = sr + slot * kSlotBytes;
@@ -457,10 +461,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ cp.async loaders
-    // Thread-issued 16-byte copies run beside the TMA engine (whose per-SM
-    // throughput alone cannot feed the tensor cores here).  Keys at or past
-    // the split end are zero-filled, so V rows the softmax masks out are exact
-    // zeros whatever the page holds.
+    // Thread-issued 16-byte copies run beside the TMA engine, whose per-SM
+    // throughput alone cannot feed the tensor cores here.
     if (ntiles > 0) {
       const int tl = threadIdx.x - 6 * 32;  // 0..63
       const int npages_valid = (kv_len + kPage - 1) / kPage;
@@ -471,27 +473,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         const int ph = p.page_table[(size_t)b * p.max_pages + pg];
         return (ph < 0 || ph >= p.num_pages) ? -1 : ph;
       };
-      int slot = 0, pos = 0, last_pos = -2;
+      int slot = 0;
       uint32_t phase = 0;
       int pend_slot[kCpDepth];
       int npend = 0, head = 0;
-      auto advance = [&]() { ++pos; if (++slot == kRing) { slot = 0; phase ^= 1; } };
+      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
+      // Copies of up to kCpDepth slots stay in flight; a slot is reported
+      // full once this thread's copies into it have landed (then made
+      // visible to the tensor cores' async proxy).  The oldest in-flight slot
+      // is at most kCpDepth - 1 < kRing positions behind the one being
+      // waited for, so no wait depends on an unreported slot.
       auto signal_oldest = [&]() {
-        const int s = pend_slot[head];
+        const int sl = pend_slot[head];
         head = (head + 1 == kCpDepth) ? 0 : head + 1;
         --npend;
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&c.fullL[s]), 0));
+        if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&c.full[sl]), 0));
       };
-      auto begin_slot = [&]() {
-        // A slot still unsignalled must never wait behind a ring position
-        // that only its own consumption can free: flush before any gap.
-        if (npend > 0 && pos != last_pos + 1) {
-          asm volatile("cp.async.wait_group 0;" ::: "memory");
-          while (npend > 0) signal_oldest();
-        }
-        last_pos = pos;
+      auto begin_slot = [&]() -> bool {
         if (lane == 0) mbar_wait(&c.empty[slot], phase ^ 1, abort);
         __syncwarp();
         return !*abort;
@@ -512,49 +512,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                      ::"r"(dst), "l"(valid ? src : p.c_kv), "r"(valid ? 16 : 0) : "memory");
       };
-      for (int t = 0; t <= ntiles && !*abort; ++t) {
-        if (t < ntiles) {  // K chunks kTmaK..8 of tile t
+      bool go = true;
+      for (int t = 0; t <= ntiles && go; ++t) {
+        if (t < ntiles) {  // K chunks: box B = this CTA's second page of the tile
           const int kb = lo + t * kTileKeys;
-          const int ph0 = phys_of(kb / kPage + 2 * (int)rank);
-          const int ph1 = phys_of(kb / kPage + 2 * (int)rank + 1);
-          for (int kc = 0; kc < 9; ++kc) {
-            if (kc < kTmaK) { advance(); continue; }
-            if (!begin_slot()) break;
-            const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
-#pragma unroll 4
-            for (int k = 0; k < 16; ++k) {
-              const int cidx = tl + kLoadThreads * k;  // 1024 16-byte units
-              const int r = cidx >> 3, u = cidx & 7;   // r: key 0..127 of this CTA
-              const int ph = (r >> 6) ? ph1 : ph0;
-              const size_t krow = (size_t)(ph < 0 ? 0 : ph) * kPage + (r & 63);
-              const void* src = kc < 8 ? (const void*)(ckv + krow * kDc + kc * 64 + u * 8)
-                                       : (const void*)(kpe + krow * kDr + u * 8);
-              const uint32_t dst = sbase + (r >> 6) * kChunkBytes + (r & 63) * 128 + ((u ^ (r & 7)) << 4);
-              cp16(dst, src, ph >= 0);
+          const int ph = phys_of(kb / kPage + 2 * (int)rank + 1);
+          const size_t prow = (size_t)(ph < 0 ? 0 : ph) * kPage;
+          for (int kc = 0; kc < 9 && go; ++kc) {
+            go = begin_slot();
+            if (!go) break;
+            const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes) + kChunkBytes;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int cidx = tl + kLoadThreads * k;  // 512 16-byte units
+              const int r = cidx >> 3, u = cidx & 7;   // r: key in the page
+              const void* src = kc < 8 ? (const void*)(ckv + (prow + r) * kDc + kc * 64 + u * 8)
+                                       : (const void*)(kpe + (prow + r) * kDr + u * 8);
+              cp16(sbase + r * 128 + ((u ^ (r & 7)) << 4), src, ph >= 0);
             }
             end_slot();
           }
         }
-        if (t > 0) {  // V slots of tile t-1: [64 keys x 128 latent columns] per page and chunk
+        if (t > 0 && go) {  // V slots of tile t-1: [64 keys x 128 latent columns]
           const int kb = lo + (t - 1) * kTileKeys;
-          for (int pg = 0; pg < 4; ++pg) {
+          for (int pg = 0; pg < 4 && go; ++pg) {
             const int k0 = kb + pg * kPage;
             if (k0 >= hi) break;
+            const bool part = v_partial(k0);
             const int ph = phys_of(k0 / kPage);
-            for (int nc = 0; nc < 2; ++nc) {
-              if (!begin_slot()) break;
+            const size_t prow = (size_t)(ph < 0 ? 0 : ph) * kPage;
+            for (int nc = 0; nc < 2 && go; ++nc) {
+              go = begin_slot();
+              if (!go) break;
               const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
               const int col0 = nc * 256 + (int)rank * 128;
+              if (!part) {  // box B: latent columns col0 + 64 .. col0 + 127
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const int cidx = tl + kLoadThreads * k;
+                  const int r = cidx >> 3, u = cidx & 7;
+                  cp16(sbase + kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
+                       ckv + (prow + r) * kDc + col0 + 64 + u * 8, ph >= 0);
+                }
+              } else {  // both boxes; keys past the range become zeros
 #pragma unroll 4
-              for (int k = 0; k < 16; ++k) {
-                const int cidx = tl + kLoadThreads * k;
-                const int r = cidx >> 4, u16 = cidx & 15;  // r: key in page, u16: 16 B unit of 256 B
-                const int sub = u16 >> 3, u = u16 & 7;
-                const bool valid = ph >= 0 && k0 + r < hi;
-                const size_t krow = (size_t)(ph < 0 ? 0 : ph) * kPage + r;
-                const void* src = ckv + krow * kDc + col0 + u16 * 8;
-                const uint32_t dst = sbase + sub * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4);
-                cp16(dst, src, valid);
+                for (int k = 0; k < 16; ++k) {
+                  const int cidx = tl + kLoadThreads * k;
+                  const int r = cidx >> 4, u16 = cidx & 15;
+                  const int sub = u16 >> 3, u = u16 & 7;
+                  cp16(sbase + sub * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
+                       ckv + (prow + r) * kDc + col0 + u16 * 8, ph >= 0 && k0 + r < hi);
+                }
               }
               end_slot();
             }
