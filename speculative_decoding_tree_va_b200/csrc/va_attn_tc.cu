@@ -46,7 +46,15 @@ namespace {
 constexpr int kThreads = 256;          // 8 warps
 constexpr int kLoadWarps = 2;          // warps 6-7: cp.async loaders
 constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kCpDepth = 3;            // slots of cp.async groups in flight per loader thread
+#ifndef VA_CP_DEPTH
+#define VA_CP_DEPTH 6
+#endif
+constexpr int kCpDepth = VA_CP_DEPTH;
+#ifndef VA_USE_LOADERS
+#define VA_USE_LOADERS 0
+#endif
+// 1: every slot is half TMA, half cp.async loaders; 0: TMA only (comparison build)
+constexpr bool kLoaders = VA_USE_LOADERS != 0;  // cp.async slot groups in flight per loader thread (< 8: see the loaders)
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
 constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
@@ -119,7 +127,7 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       "selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0;
@@ -154,13 +162,17 @@ __device__ __noinline__ void settle() {
   const unsigned long long t0 = global_ns();
   while (global_ns() - t0 < 200000ull) { }
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar_cluster, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
-               ::"r"(bar_cluster), "r"(bytes) : "memory");
+// Barrier operations keep the default (CTA-scope) memory semantics.  The
+// data they publish is either written by TMA (counted by the transaction
+// bytes) or made visible to the tensor cores' async proxy by an explicit
+// proxy fence before the arrival; cluster-scope release on every arrival
+// was measured to cut the TMA stream to about a third.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar_local, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(bar_local), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-               ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 // 2-D TMA load into this CTA's shared memory, completion counted on the
 // pair leader's barrier (cta_group::2 form).  No cluster multicast.
@@ -279,7 +291,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&c.full[s], 1 + 2 * kLoadWarps);
+      mbar_init(&c.full[s], kLoaders ? 1 + 2 * kLoadWarps : 1);
       mbar_init(&c.empty[s], 1);
     }
     mbar_init(&c.q_full, 1);
@@ -313,13 +325,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   // loader warp of both CTAs are in.  V slots of a page that ends inside the
   // key range (or is invalid) are loaded entirely by the loaders, which
   // zero-fill keys past the range, so the TMA side posts no bytes for them.
-  auto v_partial = [&](int k0) -> bool { return k0 + kPage > hi; };
+  auto v_partial = [&](int k0) -> bool { return kLoaders && k0 + kPage > hi; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && ntiles > 0) {
       const uint32_t q_bar = map_to_rank(smem_u32(&c.q_full), 0);
-      if (rank == 0) mbar_arrive_expect_tx(q_bar, 2 * kQBytes);
+      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.q_full), 2 * kQBytes);
       const int qrow = b * p.R + row0;
       for (int ch = 0; ch < 8; ++ch)
         tma_load_2d(smem_u32(sQ + ch * kChunkBytes), &tm_qn, q_bar, ch * 64, qrow);
@@ -340,7 +352,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       auto acquire = [&](uint32_t bytes, uint32_t* bar) -> bool {
         if (!mbar_wait(&c.empty[slot], phase ^ 1, abort)) return false;
         *bar = map_to_rank(smem_u32(&c.full[slot]), 0);
-        if (rank == 0) mbar_arrive_expect_tx(*bar, 2 * bytes);
+        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.full[slot]), 2 * bytes);
         return true;
       };
       bool go = true;
@@ -350,10 +362,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           const int r0 = page_row(kb / kPage + 2 * (int)rank);
           for (int kc = 0; kc < 9 && go; ++kc) {
             uint32_t bar;
-            go = acquire(kChunkBytes, &bar);
+            go = acquire(kLoaders ? kChunkBytes : kSlotBytes, &bar);
             if (!go) break;
-            tma_load_2d(smem_u32(sRing + (size_t)slot * kSlotBytes), kc < 8 ? &tm_ckv : &tm_kpe,
-                        bar, kc < 8 ? kc * 64 : 0, r0);
+            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+            tma_load_2d(dst, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0, r0);
+            if (!kLoaders)
+              tma_load_2d(dst + kChunkBytes, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0,
+                          page_row(kb / kPage + 2 * (int)rank + 1));
             advance();
           }
         }
@@ -366,11 +381,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
             const int r = page_row(k0 / kPage);
             for (int nc = 0; nc < 2 && go; ++nc) {
               uint32_t bar;
-              go = acquire(part ? 0u : (uint32_t)kChunkBytes, &bar);
+              go = acquire(part ? 0u : (uint32_t)(kLoaders ? kChunkBytes : kSlotBytes), &bar);
               if (!go) break;
-              if (!part)
-                tma_load_2d(smem_u32(sRing + (size_t)slot * kSlotBytes), &tm_ckv, bar,
-                            nc * 256 + (int)rank * 128, r);
+              if (!part) {
+                const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+                tma_load_2d(dst, &tm_ckv, bar, nc * 256 + (int)rank * 128, r);
+                if (!kLoaders)
+                  tma_load_2d(dst + kChunkBytes, &tm_ckv, bar, nc * 256 + (int)rank * 128 + 64, r);
+              }
               advance();
             }
           }
@@ -463,7 +481,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     // ------------------------------------------------------------ cp.async loaders
     // Thread-issued 16-byte copies run beside the TMA engine, whose per-SM
     // throughput alone cannot feed the tensor cores here.
-    if (ntiles > 0) {
+    if (kLoaders && ntiles > 0) {
       const int tl = threadIdx.x - 6 * 32;  // 0..63
       const int npages_valid = (kv_len + kPage - 1) / kPage;
       const __nv_bfloat16* ckv = reinterpret_cast<const __nv_bfloat16*>(p.c_kv);
