@@ -419,20 +419,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       int slot = 0;
       uint32_t phase = 0;
       auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      bool ok = mbar_wait(&c.q_full, 0, abort);
+      // Descriptors are built once; a K step only adds its byte offset / 16
+      // to the start-address field (no carry: every operand lies inside the
+      // 256 KB shared window, whose addresses fit the 14-bit field).
+      const uint64_t dq0 = sw128_desc(sq, 16, 1024);           // Q, K-major
+      const uint64_t dp0 = sw128_desc(sp, 16, 1024);           // P, K-major
+      const uint64_t dk0 = sw128_desc(sr, 16, 1024);           // K slot, K-major
+      const uint64_t dv0 = sw128_desc(sr, kChunkBytes, 1024);  // V slot, MN-major
+      auto wait = [&](uint64_t* bar, uint32_t par) -> bool {  // fast path inline
+        return mbar_try(smem_u32(bar), par) || mbar_wait(bar, par, abort);
+      };
+      bool ok = wait(&c.q_full, 0);
       auto qk = [&](int t) {
         const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
         for (int kc = 0; kc < 9 && ok; ++kc) {
-          ok = mbar_wait(&c.full[slot], phase, abort);
+          ok = wait(&c.full[slot], phase);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kslot = sr + slot * kSlotBytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = sw128_desc(sq + kc * kChunkBytes + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(kslot + kk * 32, 16, 1024);
-            mma_bf16_pair(d, a, bd, kIdQK, (kc | kk) != 0);
-          }
+          const uint64_t da = dq0 + (uint64_t)((kc * kChunkBytes) >> 4);
+          const uint64_t db = dk0 + (uint64_t)((slot * kSlotBytes) >> 4);
+          mma_bf16_pair(d, da, db, kIdQK, kc != 0);
+          mma_bf16_pair(d, da + 2, db + 2, kIdQK, 1u);
+          mma_bf16_pair(d, da + 4, db + 4, kIdQK, 1u);
+          mma_bf16_pair(d, da + 6, db + 6, kIdQK, 1u);
           mma_commit_pair(&c.empty[slot]);
           advance();
         }
@@ -440,25 +449,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       };
       auto pv = [&](int t) {
         const int kb = lo + t * kTileKeys;
-        if (ok) ok = mbar_wait(&c.p_ready, t & 1, abort);
+        if (ok) ok = wait(&c.p_ready, t & 1);
         if (!ok) return;
         tc_fence_after();
         for (int pg = 0; pg < 4 && ok; ++pg) {
           if (kb + pg * kPage >= hi) break;
+          const int nk = min(4, (hi - (kb + pg * kPage) + 15) >> 4);  // 16-key steps in range
+          const uint64_t da = dp0 + (uint64_t)((pg * kChunkBytes) >> 4);
           for (int nc = 0; nc < 2 && ok; ++nc) {
-            ok = mbar_wait(&c.full[slot], phase, abort);
+            ok = wait(&c.full[slot], phase);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vslot = sr + slot * kSlotBytes;
             const uint32_t d = tmem + kTmemO + nc * 128;
-            for (int kk = 0; kk < 4; ++kk) {
-              const int k0 = kb + pg * kPage + kk * 16;
-              if (k0 >= hi) break;
-              const int ks = pg * 4 + kk;  // 16-key step inside the 256-key tile
-              const uint64_t a = sw128_desc(sp + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(vslot + kk * 2048, kChunkBytes, 1024);
-              mma_bf16_pair(d, a, bd, kIdPV, !(t == 0 && pg == 0 && kk == 0));
-            }
+            const uint64_t db = dv0 + (uint64_t)((slot * kSlotBytes) >> 4);
+            const uint32_t acc0 = (t == 0 && pg == 0) ? 0u : 1u;
+            mma_bf16_pair(d, da, db, kIdPV, acc0);
+            if (nk > 1) mma_bf16_pair(d, da + 2, db + 128, kIdPV, 1u);
+            if (nk > 2) mma_bf16_pair(d, da + 4, db + 256, kIdPV, 1u);
+            if (nk > 3) mma_bf16_pair(d, da + 6, db + 384, kIdPV, 1u);
             mma_commit_pair(&c.empty[slot]);
             advance();
           }
