@@ -54,7 +54,14 @@ constexpr int kCpDepth = VA_CP_DEPTH;
 #define VA_USE_LOADERS 0
 #endif
 // 1: every slot is half TMA, half cp.async loaders; 0: TMA only (comparison build)
-constexpr bool kLoaders = VA_USE_LOADERS != 0;  // cp.async slot groups in flight per loader thread (< 8: see the loaders)
+constexpr bool kLoaders = VA_USE_LOADERS != 0;
+#ifndef VA_PREFETCH_AHEAD
+#define VA_PREFETCH_AHEAD 2
+#endif
+// The first row tile of each request pulls the pages of key tile t + this
+// into L2 while it loads tile t, so the other row tiles of the request (which
+// stream the same pages) find them there.  0 disables.
+constexpr int kPrefetchAhead = VA_PREFETCH_AHEAD;  // cp.async slot groups in flight per loader thread (< 8: see the loaders)
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
 constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
@@ -183,6 +190,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_leader), "r"(x), "r"(y)
       : "memory");
+}
+// Pull a [64 x 64] box into L2 ahead of use (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -356,7 +368,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         return true;
       };
       bool go = true;
+      auto prefetch_tile = [&](int t) {
+        if (kPrefetchAhead == 0 || tile_m != 0 || t >= ntiles) return;
+        const int kb = lo + t * kTileKeys;
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int pg = kb / kPage + 2 * (int)rank + q2;
+          if (pg >= npages_valid || kb + (2 * (int)rank + q2) * kPage >= hi) continue;
+          const int r = page_row(pg);
+          if (r == oob_row) continue;
+          for (int ch = 0; ch < 8; ++ch) tma_prefetch_l2(&tm_ckv, ch * 64, r);
+          tma_prefetch_l2(&tm_kpe, 0, r);
+        }
+      };
+      for (int t = 0; t < kPrefetchAhead; ++t) prefetch_tile(t);
       for (int t = 0; t <= ntiles && go; ++t) {
+        prefetch_tile(t + kPrefetchAhead);
         if (t < ntiles) {  // K chunks: box A = this CTA's first page of the tile
           const int kb = lo + t * kTileKeys;
           const int r0 = page_row(kb / kPage + 2 * (int)rank);
@@ -501,7 +527,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       };
       int slot = 0;
       uint32_t phase = 0;
-      int pend_slot[kCpDepth];
+      int pend_slot[kCpDepth] = {};
       int npend = 0, head = 0;
       auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
       // Copies of up to kCpDepth slots stay in flight; a slot is reported
