@@ -56,7 +56,7 @@ constexpr int kCpDepth = VA_CP_DEPTH;
 // 1: every slot is half TMA, half cp.async loaders; 0: TMA only (comparison build)
 constexpr bool kLoaders = VA_USE_LOADERS != 0;
 #ifndef VA_PREFETCH_AHEAD
-#define VA_PREFETCH_AHEAD 2
+#define VA_PREFETCH_AHEAD 0
 #endif
 // The first row tile of each request pulls the pages of key tile t + this
 // into L2 while it loads tile t, so the other row tiles of the request (which
