@@ -193,6 +193,32 @@ int va_verify_attn(const va_attn_args* args, va_stream_t stream);
 int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,
              int out_dtype, void* out, float* lse, va_stream_t stream);
 
+/* Size of the fixed device array va_verify_attn_noalloc keeps its split-KV
+ * partials in (on every device that loads the library, until exit). */
+#define VA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * va_verify_attn without a caller-provided workspace.  The pages have no
+ * counterpart of this call: it exists for callers that cannot allocate device
+ * memory when they run the verify step -- a serving loop whose device memory
+ * is planned once at start-up, or a latency-critical path where an
+ * allocation, which may synchronise the device, is not acceptable.
+ *
+ * Same arguments, checks, split plan and results as va_verify_attn, except
+ * that args->workspace / workspace_bytes are ignored: the split-KV partials
+ * live in a fixed array of VA_NOALLOC_SCRATCH_BYTES inside the library.
+ *   - Returns VA_ERR_UNSUPPORTED, before launching anything, when the
+ *     partials need more than that: S * B * T * H * (512 + 1) floats (each
+ *     part rounded up to 256 bytes) must fit.  S = 1 needs no scratch.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the array and leaves its contents behind; calls whose
+ *     GPU work overlaps (for instance on two streams) race on it.
+ */
+int va_verify_attn_noalloc(const va_attn_args* args, va_stream_t stream);
+
 /*
  * Diagnostic: number of bounded barrier waits inside the tensor-core kernel
  * that expired on the current device since the library was loaded (each

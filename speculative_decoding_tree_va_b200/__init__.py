@@ -25,7 +25,8 @@ D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",
            "va_workspace_bytes", "va_num_splits", "va_verify_attn", "va_merge",
-           "va_device_timeouts")
+           "va_device_timeouts", "va_verify_attn_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class VaAttnArgs(ctypes.Structure):
@@ -76,6 +77,8 @@ def load_library(path: Optional[str] = None):
     lib.va_merge.argtypes = [V, V, I, I, I, I, I, V, V, V]
     lib.va_merge.restype = I
     lib.va_device_timeouts.argtypes, lib.va_device_timeouts.restype = [], ctypes.c_uint
+    lib.va_verify_attn_noalloc.argtypes = [ctypes.POINTER(VaAttnArgs), V]
+    lib.va_verify_attn_noalloc.restype = I
     if path is None:
         _lib = lib
     return lib
@@ -190,6 +193,13 @@ def verify_attn(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, *, scal
         args.workspace, args.workspace_bytes = workspace.data_ptr(), need
     verify_attn_args(args, stream)
     return out, lse
+
+
+def verify_attn_noalloc(args: VaAttnArgs, stream=None):
+    """va_verify_attn_noalloc: split-KV partials in the library's fixed device
+    array instead of a workspace (for callers that cannot allocate)."""
+    _check(load_library().va_verify_attn_noalloc(ctypes.byref(args), _stream(stream)),
+           "va_verify_attn_noalloc")
 
 
 def merge(o_part, lse_part, out_dtype, stream=None):
