@@ -175,8 +175,9 @@ int va_num_splits(const va_attn_args* args);
  * C = ceil(ceil(kv_len / S) / 256) * 256; the partials go to the workspace
  * and va_merge combines them on the same stream.
  * bf16 runs on tensor cores with fp32 accumulation; fp32 on CUDA cores.
- * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, B >= 0, every
- * page slot below kv_len holds finite values.
+ * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, B >= 0.  Slots past
+ * kv_len in a request's last page may hold any finite values (they are
+ * multiplied by exact zeros; NaN or Inf there would propagate).
  */
 int va_verify_attn(const va_attn_args* args, va_stream_t stream);
 
