@@ -46,15 +46,16 @@ namespace {
 constexpr int kThreads = 256;          // 8 warps
 constexpr int kLoadWarps = 2;          // warps 6-7: cp.async loaders
 constexpr int kLoadThreads = 32 * kLoadWarps;
-#ifndef VA_CP_DEPTH
-#define VA_CP_DEPTH 6
-#endif
-constexpr int kCpDepth = VA_CP_DEPTH;
 #ifndef VA_USE_LOADERS
 #define VA_USE_LOADERS 0
 #endif
-// 1: every slot is half TMA, half cp.async loaders; 0: TMA only (comparison build)
-constexpr bool kLoaders = VA_USE_LOADERS != 0;
+// Second copy path beside TMA: 0 = TMA only; 1 = cp.async loader warps bring
+// box B of every V slot; 2 = box B of every slot.
+constexpr int kLoadMode = VA_USE_LOADERS;
+constexpr bool kLoaders = kLoadMode != 0;
+__host__ __device__ constexpr bool loader_box_b(bool is_v) {
+  return kLoadMode == 2 || (kLoadMode == 1 && is_v);
+}
 #ifndef VA_PREFETCH_AHEAD
 #define VA_PREFETCH_AHEAD 0
 #endif
@@ -88,7 +89,8 @@ struct TcParams {
 };
 
 struct __align__(16) Ctl {
-  uint64_t full[kRing];   // leader's expect_tx arrival + TMA bytes + loader-warp arrivals
+  uint64_t full[kRing];   // leader: expect_tx arrival + TMA bytes (+ loader threads + forwarder)
+  uint64_t fullF[kRing];  // follower: its loader threads' copies landed
   uint64_t empty[kRing];
   uint64_t q_full;
   uint64_t s_full[2];
@@ -196,6 +198,15 @@ __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, i
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
                ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
+// 3-D TMA load: coordinates (x in chunk, pool row, 64-column chunk).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
+                                            uint32_t bar_leader, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_leader), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -274,12 +285,32 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
          ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
+// Request with descending-kv_len rank `y` (ties by index).  Whole-block call.
+__device__ __noinline__ int request_of_rank(const int32_t* kv_len, int B, int y) {
+  __shared__ int found;
+  if (B > 1024) return y;  // large batches keep their natural order
+  if (threadIdx.x == 0) found = y;
+  __syncthreads();
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    const int ki = kv_len[i];
+    int rank = 0;
+    for (int j = 0; j < B; ++j) {
+      const int kj = kv_len[j];
+      rank += (kj > ki) || (kj == ki && j < i);
+    }
+    if (rank == y) found = i;
+  }
+  __syncthreads();
+  return found;
+}
+
 // -------------------------------------------------------------------- kernel
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qp,
                const __grid_constant__ CUtensorMap tm_ckv,
-               const __grid_constant__ CUtensorMap tm_kpe, const TcParams p) {
+               const __grid_constant__ CUtensorMap tm_kpe,
+               const __grid_constant__ CUtensorMap tm_ckv3, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -289,7 +320,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int b = blockIdx.y;
+  // Requests run longest first: grid row y takes the request of rank y in
+  // descending kv_len (ties by index), so the ragged tail of the launch is
+  // made of short row tiles.  Every CTA derives the same order itself.
+  const int b = request_of_rank(p.kv_len, p.B, blockIdx.y);
   const int split = blockIdx.z;
   const int tile_m = blockIdx.x >> 1;
   const int row0 = tile_m * 128 + (int)rank * 64;  // first query row of this CTA
@@ -303,7 +337,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&c.full[s], kLoaders ? 1 + 2 * kLoadWarps : 1);
+      mbar_init(&c.full[s], kLoaders ? 1 + kLoadThreads + 1 : 1);
+      mbar_init(&c.fullF[s], kLoadThreads);
       mbar_init(&c.empty[s], 1);
     }
     mbar_init(&c.q_full, 1);
@@ -388,11 +423,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           const int r0 = page_row(kb / kPage + 2 * (int)rank);
           for (int kc = 0; kc < 9 && go; ++kc) {
             uint32_t bar;
-            go = acquire(kLoaders ? kChunkBytes : kSlotBytes, &bar);
+            go = acquire(loader_box_b(false) ? kChunkBytes : kSlotBytes, &bar);
             if (!go) break;
             const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
             tma_load_2d(dst, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0, r0);
-            if (!kLoaders)
+            if (!loader_box_b(false))
               tma_load_2d(dst + kChunkBytes, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0,
                           page_row(kb / kPage + 2 * (int)rank + 1));
             advance();
@@ -407,13 +442,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
             const int r = page_row(k0 / kPage);
             for (int nc = 0; nc < 2 && go; ++nc) {
               uint32_t bar;
-              go = acquire(part ? 0u : (uint32_t)(kLoaders ? kChunkBytes : kSlotBytes), &bar);
+              go = acquire(part ? 0u : (uint32_t)(loader_box_b(true) ? kChunkBytes : kSlotBytes), &bar);
               if (!go) break;
               if (!part) {
                 const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-                tma_load_2d(dst, &tm_ckv, bar, nc * 256 + (int)rank * 128, r);
-                if (!kLoaders)
-                  tma_load_2d(dst + kChunkBytes, &tm_ckv, bar, nc * 256 + (int)rank * 128 + 64, r);
+                if (!loader_box_b(true))  // both chunks in one box: [chunk][64 rows][64 columns]
+                  tma_load_3d(dst, &tm_ckv3, bar, 0, r, nc * 4 + (int)rank * 2);
+                else
+                  tma_load_2d(dst, &tm_ckv, bar, nc * 256 + (int)rank * 128, r);
               }
               advance();
             }
@@ -438,6 +474,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     __syncwarp();
     named_arrive(2, 160);  // publishes bad_page to the epilogue
   } else if (warp == 1) {
+    if (kLoaders && rank == 1 && lane == 0 && ntiles > 0) {
+      // ---------------------------------------------------------- forwarder
+      // follower: pass "my loader copies landed" on to the leader's slot
+      int slot = 0;
+      uint32_t phase = 0;
+      bool go = true;
+      auto step = [&]() -> bool {
+        if (!mbar_wait(&c.fullF[slot], phase, abort)) return false;
+        fence_proxy_async();
+        mbar_arrive_cluster(map_to_rank(smem_u32(&c.full[slot]), 0));
+        if (++slot == kRing) { slot = 0; phase ^= 1; }
+        return true;
+      };
+      for (int t = 0; t <= ntiles && go; ++t) {
+        if (t < ntiles)
+          for (int kc = 0; kc < 9 && go; ++kc) go = step();
+        if (t > 0 && go) {
+          const int kb = lo + (t - 1) * kTileKeys;
+          for (int pg = 0; pg < 4 && go; ++pg) {
+            if (kb + pg * kPage >= hi) break;
+            go = step();
+            if (go) go = step();
+          }
+        }
+      }
+    }
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0 && ntiles > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
@@ -461,6 +523,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         for (int kc = 0; kc < 9 && ok; ++kc) {
           ok = wait(&c.full[slot], phase);
           if (!ok) break;
+          if (kLoaders) fence_proxy_async();  // loader copies -> tensor-core reads
           tc_fence_after();
           const uint64_t da = dq0 + (uint64_t)((kc * kChunkBytes) >> 4);
           const uint64_t db = dk0 + (uint64_t)((slot * kSlotBytes) >> 4);
@@ -485,6 +548,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           for (int nc = 0; nc < 2 && ok; ++nc) {
             ok = wait(&c.full[slot], phase);
             if (!ok) break;
+            if (kLoaders) fence_proxy_async();  // loader copies -> tensor-core reads
             tc_fence_after();
             const uint32_t d = tmem + kTmemO + nc * 128;
             const uint64_t db = dv0 + (uint64_t)((slot * kSlotBytes) >> 4);
@@ -513,8 +577,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ cp.async loaders
-    // Thread-issued 16-byte copies run beside the TMA engine, whose per-SM
-    // throughput alone cannot feed the tensor cores here.
+    // Thread-issued 16-byte copies beside the TMA engine.  No thread waits for
+    // its own copies: cp.async.mbarrier.arrive.noinc hands each slot's
+    // completion to the hardware, which arrives (once per loader thread) when
+    // all of the thread's earlier copies have landed -- on the leader's full
+    // barrier directly, or, in the follower, on fullF, which the follower's
+    // otherwise idle MMA lane forwards to the leader.
     if (kLoaders && ntiles > 0) {
       const int tl = threadIdx.x - 6 * 32;  // 0..63
       const int npages_valid = (kv_len + kPage - 1) / kPage;
@@ -527,37 +595,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       };
       int slot = 0;
       uint32_t phase = 0;
-      int pend_slot[kCpDepth] = {};
-      int npend = 0, head = 0;
       auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      // Copies of up to kCpDepth slots stay in flight; a slot is reported
-      // full once this thread's copies into it have landed (then made
-      // visible to the tensor cores' async proxy).  The oldest in-flight slot
-      // is at most kCpDepth - 1 < kRing positions behind the one being
-      // waited for, so no wait depends on an unreported slot.
-      auto signal_oldest = [&]() {
-        const int sl = pend_slot[head];
-        head = (head + 1 == kCpDepth) ? 0 : head + 1;
-        --npend;
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&c.full[sl]), 0));
-      };
       auto begin_slot = [&]() -> bool {
         if (lane == 0) mbar_wait(&c.empty[slot], phase ^ 1, abort);
         __syncwarp();
         return !*abort;
       };
       auto end_slot = [&]() {
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        int tail = head + npend;
-        if (tail >= kCpDepth) tail -= kCpDepth;
-        pend_slot[tail] = slot;
-        ++npend;
-        if (npend == kCpDepth) {
-          asm volatile("cp.async.wait_group %0;" ::"n"(kCpDepth - 1) : "memory");
-          signal_oldest();
-        }
+        const uint32_t bar = smem_u32(rank == 0 ? &c.full[slot] : &c.fullF[slot]);
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
         advance();
       };
       auto cp16 = [&](uint32_t dst, const void* src, bool valid) {
@@ -573,14 +619,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           for (int kc = 0; kc < 9 && go; ++kc) {
             go = begin_slot();
             if (!go) break;
-            const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes) + kChunkBytes;
+            if (loader_box_b(false)) {
+              const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes) + kChunkBytes;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int cidx = tl + kLoadThreads * k;  // 512 16-byte units
-              const int r = cidx >> 3, u = cidx & 7;   // r: key in the page
-              const void* src = kc < 8 ? (const void*)(ckv + (prow + r) * kDc + kc * 64 + u * 8)
-                                       : (const void*)(kpe + (prow + r) * kDr + u * 8);
-              cp16(sbase + r * 128 + ((u ^ (r & 7)) << 4), src, ph >= 0);
+              for (int k = 0; k < 8; ++k) {
+                const int cidx = tl + kLoadThreads * k;  // 512 16-byte units
+                const int r = cidx >> 3, u = cidx & 7;   // r: key in the page
+                const void* src = kc < 8 ? (const void*)(ckv + (prow + r) * kDc + kc * 64 + u * 8)
+                                         : (const void*)(kpe + (prow + r) * kDr + u * 8);
+                cp16(sbase + r * 128 + ((u ^ (r & 7)) << 4), src, ph >= 0);
+              }
             }
             end_slot();
           }
@@ -598,15 +646,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
               if (!go) break;
               const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
               const int col0 = nc * 256 + (int)rank * 128;
-              if (!part) {  // box B: latent columns col0 + 64 .. col0 + 127
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const int cidx = tl + kLoadThreads * k;
-                  const int r = cidx >> 3, u = cidx & 7;
-                  cp16(sbase + kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
-                       ckv + (prow + r) * kDc + col0 + 64 + u * 8, ph >= 0);
-                }
-              } else {  // both boxes; keys past the range become zeros
+              if (part) {  // both boxes; keys past the range become zeros
 #pragma unroll 4
                 for (int k = 0; k < 16; ++k) {
                   const int cidx = tl + kLoadThreads * k;
@@ -615,14 +655,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
                   cp16(sbase + sub * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
                        ckv + (prow + r) * kDc + col0 + u16 * 8, ph >= 0 && k0 + r < hi);
                 }
+              } else if (loader_box_b(true)) {  // box B: latent columns col0 + 64 .. col0 + 127
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const int cidx = tl + kLoadThreads * k;
+                  const int r = cidx >> 3, u = cidx & 7;
+                  cp16(sbase + kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
+                       ckv + (prow + r) * kDc + col0 + 64 + u * 8, ph >= 0);
+                }
               }
               end_slot();
             }
           }
         }
       }
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      while (npend > 0) signal_oldest();
+      asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -829,6 +876,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
+// c_kv as 3-D (64 columns of a chunk, pool row, chunk): a [64 x 64 x 2] box
+// lands as two consecutive swizzled [64 rows x 64 columns] chunks.
+bool encode_ckv3(CUtensorMap* map, const void* ptr, uint64_t rows) {
+  auto fn = get_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, kDc / 64};
+  cuuint64_t strides[2] = {(cuuint64_t)kDc * 2, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D bf16 map over a row-major [rows, cols] tensor with [64 x 64] boxes and
 // 128-byte swizzle (the layout the UMMA descriptors above expect).
 bool encode_2d(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
@@ -852,10 +914,11 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   const long long R = (long long)a.T * a.H;
   const long long rows_total = (long long)a.B * R;
   if (rows_total > 0x7fffffffLL) return cudaErrorNotSupported;
-  CUtensorMap tqn, tqp, tckv, tkpe;
+  CUtensorMap tqn, tqp, tckv, tkpe, tckv3;
   if (!encode_2d(&tqn, a.q_nope, rows_total, kDc) || !encode_2d(&tqp, a.q_pe, rows_total, kDr) ||
       !encode_2d(&tckv, a.c_kv, (uint64_t)a.num_pages * kPage, kDc) ||
-      !encode_2d(&tkpe, a.k_pe, (uint64_t)a.num_pages * kPage, kDr))
+      !encode_2d(&tkpe, a.k_pe, (uint64_t)a.num_pages * kPage, kDr) ||
+      !encode_ckv3(&tckv3, a.c_kv, (uint64_t)a.num_pages * kPage))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
@@ -880,7 +943,7 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   p.S = S;
   p.scale_log2 = a.scale * kLog2e;
   dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)S);
-  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, p);
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, tckv3, p);
   return cudaGetLastError();
 }
 
