@@ -51,6 +51,8 @@ def _load():
         lib.or_attention_rows.restype = None
         lib.or_merge.argtypes = [P, P, i32, i64, i32, P, P]
         lib.or_merge.restype = None
+        lib.or_tree_accept.argtypes = [P, P, P, i32, i32, P, P, P]
+        lib.or_tree_accept.restype = None
         _lib = lib
     return _lib
 
@@ -139,3 +141,19 @@ def merge(o_part: np.ndarray, lse_part: np.ndarray):
     lse = np.zeros(R, np.float64)
     lib.or_merge(_ptr(o_part), _ptr(lse_part), S, R, D, _ptr(out), _ptr(lse))
     return out, lse
+
+
+def tree_accept(parents: np.ndarray, tokens: np.ndarray, target_next: np.ndarray):
+    """Greedy accept walk: [B, T] parents/tokens/target_next -> (path [B,T], accept_len [B],
+    next_token [B])."""
+    lib = _load()
+    parents = np.ascontiguousarray(parents, np.int32)
+    tokens = np.ascontiguousarray(tokens, np.int32)
+    target_next = np.ascontiguousarray(target_next, np.int32)
+    B, T = parents.shape
+    path = np.empty((B, T), np.int32)
+    alen = np.empty(B, np.int32)
+    nxt = np.empty(B, np.int32)
+    lib.or_tree_accept(_ptr(parents), _ptr(tokens), _ptr(target_next), B, T, _ptr(path),
+                       _ptr(alen), _ptr(nxt))
+    return path, alen, nxt

@@ -235,4 +235,36 @@ void or_merge(const double* o_part, const double* lse_part, int S, int64_t rows,
   }
 }
 
+// Greedy tree accept ([MC] "The Context", item 3: follow the verified tree
+// with next-token / next-sibling pointers to find the accepted tokens).  For
+// request b, start at the root; while the target's greedy next token after
+// the current node (target_next[b][cur]) equals the token of one of cur's
+// children, move to that child (the lowest node index among equal tokens).
+// Absent nodes (parent -1 for i >= 1) are never children.  Outputs: the
+// accepted path path[b][0..n-1] (root first, rest -1), accept_len[b] = n
+// (tokens committed this step: n - 1 draft tokens plus the target's token
+// after the last accepted node), next_token[b] = target_next[b][last node].
+void or_tree_accept(const int32_t* parents, const int32_t* tokens, const int32_t* target_next,
+                    int B, int T, int32_t* path, int32_t* accept_len, int32_t* next_token) {
+  for (int b = 0; b < B; ++b) {
+    const int32_t* par = parents + static_cast<int64_t>(b) * T;
+    const int32_t* tok = tokens + static_cast<int64_t>(b) * T;
+    const int32_t* tgt = target_next + static_cast<int64_t>(b) * T;
+    int32_t* pb = path + static_cast<int64_t>(b) * T;
+    for (int i = 0; i < T; ++i) pb[i] = -1;
+    int cur = 0, n = 0;
+    pb[n++] = 0;
+    for (;;) {
+      int next = -1;
+      for (int i = cur + 1; i < T; ++i)  // children carry larger indices than their parent
+        if (par[i] == cur && tok[i] == tgt[cur]) { next = i; break; }
+      if (next < 0) break;
+      cur = next;
+      pb[n++] = cur;
+    }
+    accept_len[b] = n;
+    next_token[b] = tgt[cur];
+  }
+}
+
 }  // extern "C"

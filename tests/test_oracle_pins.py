@@ -406,3 +406,58 @@ def test_builder_equals_heapq_on_workload_trees(name):
         assert t["depth"][:t["n"]].tolist() == dep
         assert t["n"] == wl.T  # these workloads always fill the budget
         assert t["depth"].max() <= wl.max_depth
+
+
+# ---------------------------------------------------------------------------
+# greedy tree accept
+# ---------------------------------------------------------------------------
+
+def test_tree_accept_hand_worked():
+    g = json.load(open(os.path.join(GOLDEN, "tree_accept.json")))
+    par = np.array([g["parents"]], np.int32)
+    tok = np.array([g["tokens"]], np.int32)
+    for case in g["cases"]:
+        path, alen, nxt = oracle.tree_accept(par, tok, np.array([case["target_next"]], np.int32))
+        n = case["accept_len"]
+        assert alen[0] == n and nxt[0] == case["next_token"], case["name"]
+        assert path[0, :n].tolist() == case["path"] and (path[0, n:] == -1).all(), case["name"]
+
+
+def accept_bruteforce(parents, tokens, target):
+    """Deepest node whose whole root path follows the target's greedy tokens."""
+    T = len(parents)
+    best = [0]
+    for node in range(1, T):
+        if parents[node] == -1:
+            continue
+        chain = [node]
+        while parents[chain[-1]] != -1:
+            chain.append(parents[chain[-1]])
+        chain = chain[::-1]  # root first
+        if chain[0] != 0:
+            continue
+        if all(tokens[c] == target[p] for p, c in zip(chain, chain[1:])) and len(chain) > len(best):
+            best = chain
+    return best, target[best[-1]]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_tree_accept_bruteforce(seed):
+    rng = np.random.default_rng(seed)
+    inp = synth.make_inputs(synth.WORKLOADS["bf16-b64-ragged"], B=16, topk=3,
+                            seed=1000 + seed, with_tensors=False)
+    trees = oracle.build_trees(inp.lp, inp.tok, inp.wl.budget)
+    par, tok = trees["parent"], trees["token"]
+    B, T = par.shape
+    # target agrees with the first child's token with probability 0.7
+    target = rng.integers(0, 4096, size=(B, T)).astype(np.int32)
+    for b in range(B):
+        for t in range(T):
+            kids = [i for i in range(T) if par[b, i] == t]
+            if kids and rng.random() < 0.7:
+                target[b, t] = tok[b, kids[int(rng.integers(0, len(kids)))]]
+    path, alen, nxt = oracle.tree_accept(par, tok, target)
+    for b in range(B):
+        chain, nt = accept_bruteforce(list(par[b]), list(tok[b]), list(target[b]))
+        assert path[b, :alen[b]].tolist() == chain and nxt[b] == nt
+        assert alen[b] == len(chain) and (path[b, alen[b]:] == -1).all()
