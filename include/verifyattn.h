@@ -115,6 +115,28 @@ int va_build_tree(const double* lp, const int32_t* tok, int B, int L, int K, int
 int va_build_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
                        int32_t* tree_status, va_stream_t stream);
 
+/*
+ * Greedy tree accept (page "The Milestone Commit...", section "The Context",
+ * item 3: the verified tree is walked with next-token / next-sibling pointers
+ * to find the accepted tokens).
+ *
+ *   parents, tokens [device] int32 [B, T]   the draft tree (va_build_tree)
+ *   target_next     [device] int32 [B, T]   the target model's greedy token
+ *                                           after the path to each node
+ *   path            [device] int32 [B, T]   out: accepted nodes, root first,
+ *                                           then -1
+ *   accept_len      [device] int32 [B]      out: tokens committed this step
+ *                                           = accepted draft tokens + 1
+ *   next_token      [device] int32 [B]      out: target_next of the last
+ *                                           accepted node
+ * From the root, move to the child whose token equals target_next of the
+ * current node (lowest index among equal tokens) until none does.  Only
+ * links with 0 <= parent < index count; absent nodes are never accepted.
+ */
+int va_tree_accept(const int32_t* parents, const int32_t* tokens, const int32_t* target_next,
+                   int B, int T, int32_t* path, int32_t* accept_len, int32_t* next_token,
+                   va_stream_t stream);
+
 /* Arguments of va_verify_attn.  Zero-initialise, then fill. */
 typedef struct va_attn_args {
   int dtype;          /* VA_F32 (CUDA-core FFMA path) or VA_BF16 (tcgen05 path) */

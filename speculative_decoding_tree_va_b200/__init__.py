@@ -25,7 +25,7 @@ D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",
            "va_workspace_bytes", "va_num_splits", "va_verify_attn", "va_merge",
-           "va_device_timeouts", "va_verify_attn_noalloc")
+           "va_device_timeouts", "va_verify_attn_noalloc", "va_tree_accept")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -77,6 +77,8 @@ def load_library(path: Optional[str] = None):
     lib.va_merge.argtypes = [V, V, I, I, I, I, I, V, V, V]
     lib.va_merge.restype = I
     lib.va_device_timeouts.argtypes, lib.va_device_timeouts.restype = [], ctypes.c_uint
+    lib.va_tree_accept.argtypes = [V, V, V, I, I, V, V, V, V]
+    lib.va_tree_accept.restype = I
     lib.va_verify_attn_noalloc.argtypes = [ctypes.POINTER(VaAttnArgs), V]
     lib.va_verify_attn_noalloc.restype = I
     if path is None:
@@ -123,6 +125,21 @@ def build_tree(lp, tok, budget: int, stream=None):
                                         budget, _ptr(parents), _ptr(tokens), _ptr(depth),
                                         _ptr(n_nodes), _stream(stream)), "va_build_tree")
     return parents, tokens, depth, n_nodes
+
+
+def tree_accept(parents, tokens, target_next, stream=None):
+    """Greedy accept walk.  int32 [B, T] cuda tensors -> (path [B, T], accept_len [B],
+    next_token [B])."""
+    import torch
+    B, T = parents.shape
+    kw = dict(device=parents.device, dtype=torch.int32)
+    path = torch.empty(B, T, **kw)
+    alen = torch.empty(B, **kw)
+    nxt = torch.empty(B, **kw)
+    _check(load_library().va_tree_accept(_ptr(parents.contiguous()), _ptr(tokens.contiguous()),
+                                         _ptr(target_next.contiguous()), B, T, _ptr(path),
+                                         _ptr(alen), _ptr(nxt), _stream(stream)), "va_tree_accept")
+    return path, alen, nxt
 
 
 def build_tree_mask(parents, stream=None):

@@ -113,6 +113,18 @@ int va_build_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
   return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
 }
 
+int va_tree_accept(const int32_t* parents, const int32_t* tokens, const int32_t* target_next,
+                   int B, int T, int32_t* path, int32_t* accept_len, int32_t* next_token,
+                   va_stream_t stream) {
+  if (B < 0 || T < 1 || T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
+  if (B == 0) return VA_OK;
+  if (!parents || !tokens || !target_next || !path || !accept_len || !next_token)
+    return VA_ERR_INVALID_ARG;
+  cudaError_t e = va::launch_tree_accept(parents, tokens, target_next, B, T, path, accept_len,
+                                         next_token, (cudaStream_t)stream);
+  return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
+}
+
 int va_num_splits(const va_attn_args* args) {
   const int st = check_args(args);
   if (st != VA_OK) return -st;

@@ -44,6 +44,9 @@ __host__ __device__ __forceinline__ void split_range(int kv_len, int S, int s, i
 cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
                               int budget, int32_t* parents, int32_t* tokens, int32_t* depth,
                               int32_t* n_nodes, cudaStream_t st);
+cudaError_t launch_tree_accept(const int32_t* parents, const int32_t* tokens,
+                               const int32_t* target_next, int B, int T, int32_t* path,
+                               int32_t* accept_len, int32_t* next_token, cudaStream_t st);
 cudaError_t launch_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
                              int32_t* status, cudaStream_t st);
 cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float* lse_part,

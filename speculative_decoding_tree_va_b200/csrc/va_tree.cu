@@ -142,7 +142,53 @@ __global__ void tree_mask_kernel(const int32_t* __restrict__ parents, int T,
   if (i == 0 && status) status[b] = bad_any ? VA_ERR_INVALID_TREE : VA_OK;
 }
 
+// Greedy accept walk over the verified tree (page "The Milestone Commit...",
+// section "The Context", item 3: next-token / next-sibling pointers).  One
+// thread per request: link every node to its parent's child list (children
+// in increasing index order), then from the root follow the child whose
+// token equals the target's greedy next token.  Only links with
+// 0 <= parent < index count.
+__global__ void tree_accept_kernel(const int32_t* __restrict__ parents,
+                                   const int32_t* __restrict__ tokens,
+                                   const int32_t* __restrict__ target_next, int B, int T,
+                                   int32_t* __restrict__ path, int32_t* __restrict__ accept_len,
+                                   int32_t* __restrict__ next_token) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const int32_t* par = parents + (size_t)b * T;
+  const int32_t* tok = tokens + (size_t)b * T;
+  const int32_t* tgt = target_next + (size_t)b * T;
+  int32_t* pb = path + (size_t)b * T;
+  int8_t first_child[VA_MAX_QLEN], next_sib[VA_MAX_QLEN];
+  for (int i = 0; i < T; ++i) { first_child[i] = -1; next_sib[i] = -1; pb[i] = -1; }
+  for (int i = T - 1; i >= 1; --i) {
+    const int p = par[i];
+    if (p >= 0 && p < i) { next_sib[i] = first_child[p]; first_child[p] = (int8_t)i; }
+  }
+  int cur = 0, n = 0;
+  pb[n++] = 0;
+  for (;;) {
+    const int want = tgt[cur];
+    int c = first_child[cur];
+    while (c >= 0 && tok[c] != want) c = next_sib[c];
+    if (c < 0) break;
+    cur = c;
+    pb[n++] = cur;
+  }
+  accept_len[b] = n;
+  next_token[b] = tgt[cur];
+}
+
 }  // namespace
+
+cudaError_t launch_tree_accept(const int32_t* parents, const int32_t* tokens,
+                               const int32_t* target_next, int B, int T, int32_t* path,
+                               int32_t* accept_len, int32_t* next_token, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  tree_accept_kernel<<<(B + 63) / 64, 64, 0, st>>>(parents, tokens, target_next, B, T, path,
+                                                    accept_len, next_token);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
                               int budget, int32_t* parents, int32_t* tokens, int32_t* depth,
