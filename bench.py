@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 from speculative_decoding_tree_va_b200 import synth  # noqa: E402
 
 METRIC = ("verify-attn TFLOP/s & % of B200 roofline; µs per tree-verify step at B=64")
+FP32_FFMA_PEAK = 148 * 128 * 2 * 1.965e9 / 1e12  # TFLOP/s, fp32 FFMA at the max SM clock
 FLOP_PER_KEY = 2 * (synth.D_LATENT + synth.D_ROPE) + 2 * synth.D_LATENT  # QK + PV per (row, key)
 
 
@@ -42,6 +43,30 @@ def peaks():
         return m["hbm_gbs"], m["bf16_tflops"], m.get("bf16_tflops_sustained"), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def recorded_traffic(kernel_src: str, workload: str):
+    """DRAM bytes per launch of a kernel, from an ncu summary under profiles/.
+
+    A summary records them on a line
+    ``traffic-record: source_sha256=<hex> workload=<name> dram_bytes_per_launch=<int>``;
+    the figure only counts while the kernel source still hashes to <hex>."""
+    import glob
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, kernel_src), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(path) as f:
+            for line in f:
+                if not line.startswith("traffic-record:"):
+                    continue
+                kv = dict(x.split("=", 1) for x in line.split()[1:] if "=" in x)
+                if kv.get("source_sha256") == sha and kv.get("workload") == workload:
+                    return int(kv["dram_bytes_per_launch"])
+    return None
 
 
 def work(inp, depth):
@@ -263,8 +288,10 @@ def run_gpu(args):
     e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
 
     hbm, tc_peak, tc_sust, peak_src = peaks()
+    kernel_src = "speculative_decoding_tree_va_b200/csrc/" + ("va_attn_tc.cu" if bf16 else "va_attn_simt.cu")
+    traffic = recorded_traffic(kernel_src, wl.name) if S == 1 else None
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    roof_us = max(flops / (tc_peak * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
+    roof_us = max(flops / ((tc_peak if bf16 else FP32_FFMA_PEAK) * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
     clocks = clk.summary()
     if dist is not None:
         dist.destroy_process_group()
@@ -284,9 +311,12 @@ def run_gpu(args):
                    "num_splits": S, "parallelism": f"replicas x{world} (independent requests)",
                    "l2": "inputs larger than the 126 MB L2, no flush",
                    "gflop_per_step": round(flops / 1e9, 2), "alg_mb_per_step": round(alg_bytes / 1e6, 1)},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4), "traffic": None,
-                     "peak_source": f"{peak_src} bf16 dense (burst); sustained {tc_sust}",
+        "roofline": {"bound": "tensor" if bf16 else "alu", "achieved": round(achieved, 2),
+                     "peak": tc_peak if bf16 else FP32_FFMA_PEAK,
+                     "unit": "TFLOP/s", "frac": round(achieved / (tc_peak if bf16 else FP32_FFMA_PEAK), 4),
+                     "traffic": traffic,
+                     "peak_source": (f"{peak_src} bf16 dense (burst); sustained {tc_sust}" if bf16 else
+                                     "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz"),
                      "kernel": "attn_tc_kernel" if bf16 else "attn_simt_kernel",
                      "kernel_us": round(attn_ms * 1e3, 1), "roofline_us": round(roof_us, 1),
                      "frac_of_step_roofline": round(roof_us / (ms_step * 1e3), 4)},

@@ -169,6 +169,14 @@ typedef struct va_attn_args {
  * kernel (a second, independent GPU path for cross-checks). */
 #define VA_FLAG_BF16_CUDA_CORES 1
 
+/* Test hook for the bounded waits (bf16 tensor-core path only; rejected with
+ * VA_ERR_INVALID_ARG elsewhere): the kernel issues no tensor-core work, so
+ * every wait on tensor-core completion runs into its 1 s bound.  Each
+ * request then comes back with req_status VA_ERR_CUDA, zero output and lse
+ * -inf, va_device_timeouts() grows, and the context stays usable.  No copy
+ * is in flight when the CTAs give up, so nothing lands after they exit. */
+#define VA_FLAG_TEST_STALL_MMA 2
+
 /*
  * Workspace needed by va_verify_attn for these arguments (0 for a single
  * pass).  With S = the split count the call will use, the workspace holds

@@ -21,6 +21,7 @@ LIB_PATH = os.environ.get("VA_LIB", os.path.join(HERE, "libverifyattn.so"))
 VA_OK, VA_ERR_INVALID_ARG, VA_ERR_UNSUPPORTED, VA_ERR_CUDA, VA_ERR_INVALID_TREE = range(5)
 VA_F32, VA_BF16 = 0, 1
 VA_FLAG_BF16_CUDA_CORES = 1
+VA_FLAG_TEST_STALL_MMA = 2  # test hook: the tensor-core kernel's bounded waits expire
 D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",

@@ -20,7 +20,10 @@ int check_args(const va_attn_args* a) {
   if (a->B < 0 || a->H < 1 || a->T < 1 || a->T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
   if (a->page_size != VA_PAGE_SIZE) return VA_ERR_UNSUPPORTED;
   if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
-  if (a->flags & ~VA_FLAG_BF16_CUDA_CORES) return VA_ERR_INVALID_ARG;
+  if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA)) return VA_ERR_INVALID_ARG;
+  if ((a->flags & VA_FLAG_TEST_STALL_MMA) &&
+      (a->dtype != VA_BF16 || (a->flags & VA_FLAG_BF16_CUDA_CORES)))
+    return VA_ERR_INVALID_ARG;  // only the tensor-core kernel has the hook
   if (!(a->scale == a->scale)) return VA_ERR_INVALID_ARG;  // NaN scale
   if (a->B == 0) return VA_OK;
   if (a->num_pages < 1 || a->max_pages < 1) return VA_ERR_INVALID_ARG;

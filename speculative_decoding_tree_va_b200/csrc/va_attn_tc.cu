@@ -85,6 +85,7 @@ struct TcParams {
   float* lse_part;
   int32_t* req_status;
   int B, H, T, R, max_pages, num_pages, S;
+  int stall_mma;  // test hook: issue no tensor-core work (the waits expire)
   float scale_log2;
 };
 
@@ -102,6 +103,7 @@ struct __align__(16) Ctl {
   int bad_page;
   float xmax[2][2][64];  // [tile parity][column half][row]
   float xsum[2][64];
+  float xsumr[2][64];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kPBytes + (size_t)kRing * kSlotBytes + sizeof(Ctl);
@@ -501,7 +503,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       }
     }
     // ------------------------------------------------------------ MMA issuer
-    if (rank == 0 && lane == 0 && ntiles > 0) {
+    if (rank == 0 && lane == 0 && ntiles > 0 && !p.stall_mma) {
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
       const uint32_t sq = smem_u32(sQ), sp = smem_u32(sP), sr = smem_u32(sRing);
       int slot = 0;
@@ -690,7 +692,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       live = mask_bit(mrow, t);
     }
     const uint32_t p_ready_leader = map_to_rank(smem_u32(&c.p_ready), 0);
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f, lr = 0.f;  // lr: sum of the bf16-rounded probabilities
 
     for (int t = 0; t < ntiles; ++t) {
       const int kb = lo + t * kTileKeys;
@@ -736,7 +738,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         m_used = tmax;
       }
       uint32_t pk[64];
-      float sum = 0.f;
+      float sum = 0.f, sumr = 0.f;
       if (m_used == -INFINITY) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) pk[i] = 0u;
@@ -747,9 +749,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           const float p1 = exp2f(x[2 * i + 1] - m_used);
           sum += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
+          sumr += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
         }
       }
       l = l * alpha + sum;
+      lr = lr * alpha + sumr;
 
       // PV(t-1) must be done before P is overwritten or O rescaled
       if (t > 0) {
@@ -794,12 +798,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       tc_fence_after();
     }
     c.xsum[h][m] = l;
+    c.xsumr[h][m] = lr;
     named_sync(1, 128);
     named_sync(2, 160);
     const float lsum = l + c.xsum[h ^ 1][m];
+    const float lsumr = lr + c.xsumr[h ^ 1][m];
     const bool bad = !req_ok || c.bad_page || *abort;
-    const bool empty = bad || !(lsum > 0.f) || ntiles == 0;
-    const float inv = empty ? 0.f : 1.f / lsum;
+    const bool empty = bad || !(lsum > 0.f) || !(lsumr > 0.f) || ntiles == 0;
+    const float inv = empty ? 0.f : 1.f / lsumr;
     const float lse = empty ? -INFINITY : (m_used + log2f(lsum)) * kLn2;
     __syncwarp();
     {
@@ -941,6 +947,7 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   p.max_pages = a.max_pages;
   p.num_pages = a.num_pages;
   p.S = S;
+  p.stall_mma = (a.flags & VA_FLAG_TEST_STALL_MMA) ? 1 : 0;
   p.scale_log2 = a.scale * kLog2e;
   dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)S);
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, tckv3, p);

@@ -140,6 +140,23 @@ def test_values_beyond_kv_len_do_not_leak(va, dtype, path):
 
 
 @pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
+def test_poisoned_request_stays_contained(va, dtype, path):
+    """NaN in one request's queries and +inf in its keys reach no other request."""
+    inp = edge_inputs(dtype, B=3, H=8, P=(70, 400), budget=12)
+    nan_, inf_ = (np.uint16(0x7FC0), np.uint16(0x7F80)) if dtype == "bf16" else (np.nan, np.inf)
+    inp.q_nope[0, 1, 2, 5] = nan_
+    inp.c_kv[inp.page_table[0, 0], 3, 7] = inf_
+    inp.k_pe[inp.page_table[0, 1], 9, 2] = inf_
+    parents = trees_for(inp)["parent"]
+    out, lse, mask = run_gpu(va, inp, parents, path)
+    R = inp.T * inp.wl.H
+    rows = np.arange(R, 3 * R, dtype=np.int32)
+    ref_out, ref_lse = oracle_rows(inp, mask, rows=rows)
+    compare(out[R:], lse[R:], ref_out, ref_lse, dtype, "requests 1-2")
+    assert not np.isfinite(out[:R]).all()   # the poisoned request does see its own inputs
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
 def test_bad_kv_len_and_page_are_flagged(va, dtype, path):
     import torch
     inp = edge_inputs(dtype, B=3, H=8, P=(70, 200), budget=8)

@@ -1,0 +1,49 @@
+"""Failure detection on the GPU without a fault: the tensor-core kernel's
+barrier waits are bounded, and an expired wait comes back as a status.
+
+VA_FLAG_TEST_STALL_MMA makes the kernel issue no tensor-core work, so every
+wait on tensor-core completion runs into its 1 s bound (a flag that nothing
+sets).  The test checks the per-request status, the output of flagged rows,
+the timeout counter, and that the same context then runs a normal call."""
+import numpy as np
+import pytest
+
+from speculative_decoding_tree_va_b200 import synth
+from _harness import compare, oracle_rows, to_device, trees_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def va():
+    import torch
+    assert torch.cuda.is_available()
+    import speculative_decoding_tree_va_b200 as m
+    m.load_library()
+    return m
+
+
+def test_expired_waits_flag_requests_and_leave_the_context_usable(va):
+    import torch
+    inp = synth.make_inputs(synth.WORKLOADS["bf16-deep"], B=2, H=16, P=(100, 300), budget=8)
+    d = to_device(inp, trees_for(inp)["parent"])
+    mask, _ = va.build_tree_mask(d["parents"])
+    call = dict(scale=synth.SCALE, num_splits=1)
+    before = va.device_timeouts()
+    st = torch.zeros(inp.wl.B, dtype=torch.int32, device="cuda")
+    out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
+                              d["kv_len"], mask, req_status=st, flags=va.VA_FLAG_TEST_STALL_MMA,
+                              **call)
+    torch.cuda.synchronize()
+    assert st.cpu().tolist() == [va.VA_ERR_CUDA] * inp.wl.B
+    assert torch.isneginf(lse).all() and not out.float().abs().sum()
+    assert va.device_timeouts() > before
+
+    st.zero_()
+    out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
+                              d["kv_len"], mask, req_status=st, **call)
+    torch.cuda.synchronize()
+    assert st.cpu().tolist() == [0] * inp.wl.B
+    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64))
+    compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+            ref_out, ref_lse, "bf16", "after the stalled call")
