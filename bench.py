@@ -139,28 +139,52 @@ class Clocks:
                 "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU under torchrun: (rank, local rank, torch.distributed or None).
+
+    `backend` is "nccl" on GPUs; the rank plumbing is tested with "gloo" on CPU."""
     import torch
     import torch.distributed as dist
     if n_gpus > 1:
+        import datetime
         rank = int(os.environ["RANK"])
         local = int(os.environ.get("LOCAL_RANK", rank))
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
         return rank, local, dist
-    torch.cuda.set_device(0)
+    if backend == "nccl":
+        torch.cuda.set_device(0)
     return 0, 0, None
 
 
-def max_over_ranks(x: float, dist) -> float:
+def max_over_ranks(x: float, dist, device="cuda") -> float:
+    """The slowest rank's figure (every rank takes part; all get the same value)."""
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(wl, rank: int) -> int:
+    """Each rank verifies its own independent batch (weak scaling)."""
+    return wl.seed + 7919 * rank
+
+
+def config_of(wl, S, world, flops, alg_bytes):
+    """The workload description both arms print."""
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T,
+            "prefix": list(wl.P) if isinstance(wl.P, tuple) else wl.P,
+            "tree": f"best-first top-{wl.topk}, depth<={wl.max_depth}, budget {wl.budget}",
+            "kv": "64-token pages, shuffled" if wl.paged else "contiguous",
+            "num_splits": S, "parallelism": f"replicas x{world} (independent requests)",
+            "l2": ("inputs larger than the 126 MB L2, no flush" if alg_bytes > 126e6 else
+                   "inputs fit in the 126 MB L2 and are not flushed (warm-cache figure)"),
+            "gflop_per_step": round(flops / 1e9, 2), "alg_mb_per_step": round(alg_bytes / 1e6, 1)}
 
 
 def run_gpu(args):
@@ -170,7 +194,7 @@ def run_gpu(args):
     rank, local, dist = dist_setup(args.gpus)
     wl = synth.WORKLOADS[args.workload]
     # every rank verifies its own batch (independent requests): weak scaling
-    inp = synth.make_inputs(wl, seed=wl.seed + 7919 * rank)
+    inp = synth.make_inputs(wl, seed=rank_seed(wl, rank))
     dev = torch.device("cuda", local)
     bf16 = wl.dtype == "bf16"
     tdt = torch.bfloat16 if bf16 else torch.float32
@@ -304,13 +328,7 @@ def run_gpu(args):
         "us_per_step": round(ms_step * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded; no dataset or weights)",
-        "config": {"workload": wl.name, "B": B, "H": H, "T": T,
-                   "prefix": list(wl.P) if isinstance(wl.P, tuple) else wl.P,
-                   "tree": f"best-first top-{wl.topk}, depth<={wl.max_depth}, budget {wl.budget}",
-                   "kv": "64-token pages, shuffled" if wl.paged else "contiguous",
-                   "num_splits": S, "parallelism": f"replicas x{world} (independent requests)",
-                   "l2": "inputs larger than the 126 MB L2, no flush",
-                   "gflop_per_step": round(flops / 1e9, 2), "alg_mb_per_step": round(alg_bytes / 1e6, 1)},
+        "config": config_of(wl, S, world, flops, alg_bytes),
         "roofline": {"bound": "tensor" if bf16 else "alu", "achieved": round(achieved, 2),
                      "peak": tc_peak if bf16 else FP32_FFMA_PEAK,
                      "unit": "TFLOP/s", "frac": round(achieved / (tc_peak if bf16 else FP32_FFMA_PEAK), 4),
@@ -370,15 +388,17 @@ def run_reference(args):
         cpu_baseline(inp, depth, budget_s=0.2)
     vals = [cpu_baseline(inp, depth, budget_s=per_step) for _ in range(args.steps)]
     v = float(np.mean([x["value"] for x in vals]))
-    flops, _ = work(inp, depth)
+    flops, alg_bytes = work(inp, depth)
     ms = flops / (v * 1e12) * 1e3
+    S = args.splits if getattr(args, "splits", None) is not None else wl.splits
+    cfg = config_of(wl, S, args.gpus, flops, alg_bytes)
+    cfg["note"] = "each step = a bounded row sample; per-step time extrapolated per flop"
     line = {
         "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; no dataset or weights)", "impl": "reference",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T,
-                   "note": "each step = a bounded row sample; per-step time extrapolated per flop"},
+        "config": cfg,
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                          "sample": vals[0]["sample"]},
         "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
