@@ -111,6 +111,7 @@ def edge_inputs(dtype, B=2, H=8, P=0, budget=8, topk=8, max_depth=15, seed=5):
     dict(P=257, budget=64, topk=2, H=64, B=1),
     dict(P=100, budget=10, H=1),
     dict(P=(60, 70), budget=33, H=3, B=3),
+    dict(P=(1, 300), budget=0, H=1, B=1100, max_depth=1),  # more requests than the kernel ranks
 ])
 def test_edge_cases(va, dtype, path, case):
     inp = edge_inputs(dtype, **case)
