@@ -51,7 +51,7 @@ class Workload:
     topk: int                     # drafter top-k per depth
     max_depth: int = MAX_DEPTH
     paged: bool = True            # shuffled 64-token pages (else identity table)
-    splits: int = 1               # split-KV chunks for the flash-decode path
+    splits: int = 1               # split-KV chunks for the flash-decode path (0: the library plans)
     seed_index: int = 0
 
     @property
@@ -67,7 +67,7 @@ WORKLOADS = {
     "fp32-tiny": Workload("fp32-tiny", "f32", B=1, H=8, P=128, budget=8, topk=8,
                           paged=False, seed_index=0),
     "fp32-page-test": Workload("fp32-page-test", "f32", B=1, H=64, P=2048, budget=32,
-                               topk=8, paged=False, seed_index=1),
+                               topk=8, paged=False, splits=0, seed_index=1),
     "bf16-deep": Workload("bf16-deep", "bf16", B=16, H=64, P=4096, budget=64, topk=2,
                           paged=True, seed_index=2),
     "bf16-b64-ragged": Workload("bf16-b64-ragged", "bf16", B=64, H=64, P=(512, 8192),
