@@ -43,26 +43,7 @@ __device__ unsigned int g_tc_timeouts = 0;  // count of barrier waits that expir
 
 namespace {
 
-constexpr int kThreads = 256;          // 8 warps
-constexpr int kLoadWarps = 2;          // warps 6-7: cp.async loaders
-constexpr int kLoadThreads = 32 * kLoadWarps;
-#ifndef VA_USE_LOADERS
-#define VA_USE_LOADERS 0
-#endif
-// Second copy path beside TMA: 0 = TMA only; 1 = cp.async loader warps bring
-// box B of every V slot; 2 = box B of every slot.
-constexpr int kLoadMode = VA_USE_LOADERS;
-constexpr bool kLoaders = kLoadMode != 0;
-__host__ __device__ constexpr bool loader_box_b(bool is_v) {
-  return kLoadMode == 2 || (kLoadMode == 1 && is_v);
-}
-#ifndef VA_PREFETCH_AHEAD
-#define VA_PREFETCH_AHEAD 0
-#endif
-// The first row tile of each request pulls the pages of key tile t + this
-// into L2 while it loads tile t, so the other row tiles of the request (which
-// stream the same pages) find them there.  0 disables.
-constexpr int kPrefetchAhead = VA_PREFETCH_AHEAD;  // cp.async slot groups in flight per loader thread (< 8: see the loaders)
+constexpr int kThreads = 192;          // 6 warps
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
 constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
@@ -90,8 +71,7 @@ struct TcParams {
 };
 
 struct __align__(16) Ctl {
-  uint64_t full[kRing];   // leader: expect_tx arrival + TMA bytes (+ loader threads + forwarder)
-  uint64_t fullF[kRing];  // follower: its loader threads' copies landed
+  uint64_t full[kRing];   // leader: expect_tx arrival + both CTAs' TMA bytes
   uint64_t empty[kRing];
   uint64_t q_full;
   uint64_t s_full[2];
@@ -194,11 +174,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_leader), "r"(x), "r"(y)
       : "memory");
-}
-// Pull a [64 x 64] box into L2 ahead of use (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
 // 3-D TMA load: coordinates (x in chunk, pool row, 64-column chunk).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
@@ -339,8 +314,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&c.full[s], kLoaders ? 1 + kLoadThreads + 1 : 1);
-      mbar_init(&c.fullF[s], kLoadThreads);
+      mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
     mbar_init(&c.q_full, 1);
@@ -364,17 +338,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   const uint32_t tmem = c.tmem_base;
   volatile int* abort = &c.abort;
 
-  // Ring protocol.  Every 16 KB slot is two 8 KB boxes: box A comes by TMA,
-  // box B by the cp.async loader warps, so both copy engines of the SM work on
-  // every slot.  Each producer and the MMA issuer walk the same slot sequence
-  // -- for tile t: K chunks kc = 0..8 of tile t, then the V slots of tile t-1 --
-  // so every ring position is taken by each of them in order and a barrier
-  // phase can never be waited on twice ahead.  A slot is full when the
-  // leader's expect_tx arrival, both CTAs' TMA bytes and one arrival per
-  // loader warp of both CTAs are in.  V slots of a page that ends inside the
-  // key range (or is invalid) are loaded entirely by the loaders, which
-  // zero-fill keys past the range, so the TMA side posts no bytes for them.
-  auto v_partial = [&](int k0) -> bool { return kLoaders && k0 + kPage > hi; };
+  // Ring protocol.  Every 16 KB slot is two 8 KB TMA boxes (K: one per page;
+  // V: one 3-D box).  The producer and the MMA issuer walk the same slot
+  // sequence -- for tile t: K chunks kc = 0..8 of tile t, then the V slots of
+  // tile t-1 -- so every ring position is taken by both in order and a
+  // barrier phase can never be waited on twice ahead.  A slot is full when
+  // the leader's expect_tx arrival and both CTAs' TMA bytes are in.
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -405,54 +374,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         return true;
       };
       bool go = true;
-      auto prefetch_tile = [&](int t) {
-        if (kPrefetchAhead == 0 || tile_m != 0 || t >= ntiles) return;
-        const int kb = lo + t * kTileKeys;
-        for (int q2 = 0; q2 < 2; ++q2) {
-          const int pg = kb / kPage + 2 * (int)rank + q2;
-          if (pg >= npages_valid || kb + (2 * (int)rank + q2) * kPage >= hi) continue;
-          const int r = page_row(pg);
-          if (r == oob_row) continue;
-          for (int ch = 0; ch < 8; ++ch) tma_prefetch_l2(&tm_ckv, ch * 64, r);
-          tma_prefetch_l2(&tm_kpe, 0, r);
-        }
-      };
-      for (int t = 0; t < kPrefetchAhead; ++t) prefetch_tile(t);
       for (int t = 0; t <= ntiles && go; ++t) {
-        prefetch_tile(t + kPrefetchAhead);
-        if (t < ntiles) {  // K chunks: box A = this CTA's first page of the tile
+        if (t < ntiles) {  // K chunks: this CTA's two pages of the tile
           const int kb = lo + t * kTileKeys;
           const int r0 = page_row(kb / kPage + 2 * (int)rank);
+          const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
           for (int kc = 0; kc < 9 && go; ++kc) {
             uint32_t bar;
-            go = acquire(loader_box_b(false) ? kChunkBytes : kSlotBytes, &bar);
+            go = acquire(kSlotBytes, &bar);
             if (!go) break;
             const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-            tma_load_2d(dst, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0, r0);
-            if (!loader_box_b(false))
-              tma_load_2d(dst + kChunkBytes, kc < 8 ? &tm_ckv : &tm_kpe, bar, kc < 8 ? kc * 64 : 0,
-                          page_row(kb / kPage + 2 * (int)rank + 1));
+            const CUtensorMap* map = kc < 8 ? &tm_ckv : &tm_kpe;
+            const int x0 = kc < 8 ? kc * 64 : 0;
+            tma_load_2d(dst, map, bar, x0, r0);
+            tma_load_2d(dst + kChunkBytes, map, bar, x0, r1);
             advance();
           }
         }
-        if (t > 0 && go) {  // V slots of tile t-1: box A = the first 64 latent columns
+        if (t > 0 && go) {  // V slots of tile t-1: [64 keys x 2 chunks x 64 latent columns]
           const int kb = lo + (t - 1) * kTileKeys;
           for (int pg = 0; pg < 4 && go; ++pg) {
             const int k0 = kb + pg * kPage;
             if (k0 >= hi) break;
-            const bool part = v_partial(k0);
             const int r = page_row(k0 / kPage);
             for (int nc = 0; nc < 2 && go; ++nc) {
               uint32_t bar;
-              go = acquire(part ? 0u : (uint32_t)(loader_box_b(true) ? kChunkBytes : kSlotBytes), &bar);
+              go = acquire(kSlotBytes, &bar);
               if (!go) break;
-              if (!part) {
-                const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-                if (!loader_box_b(true))  // both chunks in one box: [chunk][64 rows][64 columns]
-                  tma_load_3d(dst, &tm_ckv3, bar, 0, r, nc * 4 + (int)rank * 2);
-                else
-                  tma_load_2d(dst, &tm_ckv, bar, nc * 256 + (int)rank * 128, r);
-              }
+              tma_load_3d(smem_u32(sRing + (size_t)slot * kSlotBytes), &tm_ckv3, bar, 0, r,
+                          nc * 4 + (int)rank * 2);
               advance();
             }
           }
@@ -476,32 +426,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     __syncwarp();
     named_arrive(2, 160);  // publishes bad_page to the epilogue
   } else if (warp == 1) {
-    if (kLoaders && rank == 1 && lane == 0 && ntiles > 0) {
-      // ---------------------------------------------------------- forwarder
-      // follower: pass "my loader copies landed" on to the leader's slot
-      int slot = 0;
-      uint32_t phase = 0;
-      bool go = true;
-      auto step = [&]() -> bool {
-        if (!mbar_wait(&c.fullF[slot], phase, abort)) return false;
-        fence_proxy_async();
-        mbar_arrive_cluster(map_to_rank(smem_u32(&c.full[slot]), 0));
-        if (++slot == kRing) { slot = 0; phase ^= 1; }
-        return true;
-      };
-      for (int t = 0; t <= ntiles && go; ++t) {
-        if (t < ntiles)
-          for (int kc = 0; kc < 9 && go; ++kc) go = step();
-        if (t > 0 && go) {
-          const int kb = lo + (t - 1) * kTileKeys;
-          for (int pg = 0; pg < 4 && go; ++pg) {
-            if (kb + pg * kPage >= hi) break;
-            go = step();
-            if (go) go = step();
-          }
-        }
-      }
-    }
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0 && ntiles > 0 && !p.stall_mma) {
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
@@ -525,7 +449,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         for (int kc = 0; kc < 9 && ok; ++kc) {
           ok = wait(&c.full[slot], phase);
           if (!ok) break;
-          if (kLoaders) fence_proxy_async();  // loader copies -> tensor-core reads
           tc_fence_after();
           const uint64_t da = dq0 + (uint64_t)((kc * kChunkBytes) >> 4);
           const uint64_t db = dk0 + (uint64_t)((slot * kSlotBytes) >> 4);
@@ -550,7 +473,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           for (int nc = 0; nc < 2 && ok; ++nc) {
             ok = wait(&c.full[slot], phase);
             if (!ok) break;
-            if (kLoaders) fence_proxy_async();  // loader copies -> tensor-core reads
             tc_fence_after();
             const uint32_t d = tmem + kTmemO + nc * 128;
             const uint64_t db = dv0 + (uint64_t)((slot * kSlotBytes) >> 4);
@@ -576,102 +498,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         mma_commit_pair(&c.mma_drain);
         mbar_wait_final(&c.mma_drain, 0);
       }
-    }
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------ cp.async loaders
-    // Thread-issued 16-byte copies beside the TMA engine.  No thread waits for
-    // its own copies: cp.async.mbarrier.arrive.noinc hands each slot's
-    // completion to the hardware, which arrives (once per loader thread) when
-    // all of the thread's earlier copies have landed -- on the leader's full
-    // barrier directly, or, in the follower, on fullF, which the follower's
-    // otherwise idle MMA lane forwards to the leader.
-    if (kLoaders && ntiles > 0) {
-      const int tl = threadIdx.x - 6 * 32;  // 0..63
-      const int npages_valid = (kv_len + kPage - 1) / kPage;
-      const __nv_bfloat16* ckv = reinterpret_cast<const __nv_bfloat16*>(p.c_kv);
-      const __nv_bfloat16* kpe = reinterpret_cast<const __nv_bfloat16*>(p.k_pe);
-      auto phys_of = [&](int pg) -> int {
-        if (pg >= npages_valid) return -1;
-        const int ph = p.page_table[(size_t)b * p.max_pages + pg];
-        return (ph < 0 || ph >= p.num_pages) ? -1 : ph;
-      };
-      int slot = 0;
-      uint32_t phase = 0;
-      auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      auto begin_slot = [&]() -> bool {
-        if (lane == 0) mbar_wait(&c.empty[slot], phase ^ 1, abort);
-        __syncwarp();
-        return !*abort;
-      };
-      auto end_slot = [&]() {
-        const uint32_t bar = smem_u32(rank == 0 ? &c.full[slot] : &c.fullF[slot]);
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-        advance();
-      };
-      auto cp16 = [&](uint32_t dst, const void* src, bool valid) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                     ::"r"(dst), "l"(valid ? src : p.c_kv), "r"(valid ? 16 : 0) : "memory");
-      };
-      bool go = true;
-      for (int t = 0; t <= ntiles && go; ++t) {
-        if (t < ntiles) {  // K chunks: box B = this CTA's second page of the tile
-          const int kb = lo + t * kTileKeys;
-          const int ph = phys_of(kb / kPage + 2 * (int)rank + 1);
-          const size_t prow = (size_t)(ph < 0 ? 0 : ph) * kPage;
-          for (int kc = 0; kc < 9 && go; ++kc) {
-            go = begin_slot();
-            if (!go) break;
-            if (loader_box_b(false)) {
-              const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes) + kChunkBytes;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int cidx = tl + kLoadThreads * k;  // 512 16-byte units
-                const int r = cidx >> 3, u = cidx & 7;   // r: key in the page
-                const void* src = kc < 8 ? (const void*)(ckv + (prow + r) * kDc + kc * 64 + u * 8)
-                                         : (const void*)(kpe + (prow + r) * kDr + u * 8);
-                cp16(sbase + r * 128 + ((u ^ (r & 7)) << 4), src, ph >= 0);
-              }
-            }
-            end_slot();
-          }
-        }
-        if (t > 0 && go) {  // V slots of tile t-1: [64 keys x 128 latent columns]
-          const int kb = lo + (t - 1) * kTileKeys;
-          for (int pg = 0; pg < 4 && go; ++pg) {
-            const int k0 = kb + pg * kPage;
-            if (k0 >= hi) break;
-            const bool part = v_partial(k0);
-            const int ph = phys_of(k0 / kPage);
-            const size_t prow = (size_t)(ph < 0 ? 0 : ph) * kPage;
-            for (int nc = 0; nc < 2 && go; ++nc) {
-              go = begin_slot();
-              if (!go) break;
-              const uint32_t sbase = smem_u32(sRing + (size_t)slot * kSlotBytes);
-              const int col0 = nc * 256 + (int)rank * 128;
-              if (part) {  // both boxes; keys past the range become zeros
-#pragma unroll 4
-                for (int k = 0; k < 16; ++k) {
-                  const int cidx = tl + kLoadThreads * k;
-                  const int r = cidx >> 4, u16 = cidx & 15;
-                  const int sub = u16 >> 3, u = u16 & 7;
-                  cp16(sbase + sub * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
-                       ckv + (prow + r) * kDc + col0 + u16 * 8, ph >= 0 && k0 + r < hi);
-                }
-              } else if (loader_box_b(true)) {  // box B: latent columns col0 + 64 .. col0 + 127
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const int cidx = tl + kLoadThreads * k;
-                  const int r = cidx >> 3, u = cidx & 7;
-                  cp16(sbase + kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4),
-                       ckv + (prow + r) * kDc + col0 + 64 + u * 8, ph >= 0);
-                }
-              }
-              end_slot();
-            }
-          }
-        }
-      }
-      asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
