@@ -91,6 +91,30 @@ def test_split_kv_matches_unsplit_oracle(va, path, S):
     check_full(va, inp, path, num_splits=S)
 
 
+@pytest.mark.parametrize("path", ["f32"] + BF16_PATHS)
+def test_planner_chosen_splits_match_the_oracle(va, path):
+    """num_splits = 0: the library picks the split count (and the caller's workspace size)."""
+    import torch
+    name = "fp32-page-test" if path == "f32" else "bf16-long-prefix"
+    inp = synth.make_inputs(synth.WORKLOADS[name], B=1, H=16, P=6000)
+    parents = trees_for(inp)["parent"]
+    d = to_device(inp, parents)
+    mask, _ = va.build_tree_mask(d["parents"])
+    flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
+    out = torch.empty(*d["q_nope"].shape, dtype=d["q_nope"].dtype, device="cuda")
+    lse = torch.empty(*d["q_nope"].shape[:3], dtype=torch.float32, device="cuda")
+    args = va.make_args(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"], d["kv_len"],
+                        mask, out, lse, scale=synth.SCALE, num_splits=0, flags=flags)
+    S = va.num_splits(args)
+    assert S > 1  # one request of 6000 keys leaves most SMs idle without a split
+    out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
+                              d["kv_len"], mask, scale=synth.SCALE, num_splits=0, flags=flags)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64))
+    compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+            ref_out, ref_lse, inp.wl.dtype, f"{path}, {S} planned splits")
+
+
 # --- edge cases ----------------------------------------------------------------
 
 def edge_inputs(dtype, B=2, H=8, P=0, budget=8, topk=8, max_depth=15, seed=5):
