@@ -104,3 +104,17 @@ def test_split_planning_and_workspace(lib):
     s = lib.va_num_splits(ctypes.byref(args(B=4, T=65, max_pages=2050)))
     assert s > 1 and (4 * 33 * s) % 74 >= 0
     assert lib.va_num_splits(ctypes.byref(args(T=66))) == -va.VA_ERR_INVALID_ARG
+
+
+def test_c99_program_uses_the_host_api(tmp_path):
+    """The header is plain C99 and the library links into a C program with no Python."""
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "speculative_decoding_tree_va_b200")
+    exe = str(tmp_path / "va_host_checks")
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c", "va_host_checks.c"),
+                    "-L", pkg, "-lverifyattn", "-Wl,-rpath," + pkg, "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "host checks ok" in r.stdout
