@@ -358,7 +358,11 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank != 0:
         return
-    cpu = None if args.no_cpu_baseline else cpu_baseline(inp, depth_h, budget_s=args.cpu_seconds)
+    cpu = None
+    if not args.no_cpu_baseline:
+        gpu_out = out.float().cpu().numpy().reshape(-1, synth.D_LATENT)
+        gpu_lse = lse.cpu().numpy().reshape(-1)
+        cpu = cpu_baseline(inp, depth_h, budget_s=args.cpu_seconds, gpu_out=gpu_out, gpu_lse=gpu_lse)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -385,8 +389,25 @@ def run_gpu(args):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(inp, depth, budget_s=15.0):
-    """fp64 oracle, single-threaded, on a seeded sample of whole rows."""
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count(), model
+
+
+def cpu_baseline(inp, depth, budget_s=15.0, gpu_out=None, gpu_lse=None):
+    """fp64 oracle, single-threaded, on a seeded sample of whole rows.
+
+    With the GPU's out / lse of the same workload (host numpy arrays, one row per
+    (b, t, h)), the sampled rows are also compared with it element by element."""
     import oracle
     B, T, H = inp.wl.B, inp.T, inp.wl.H
     trees = oracle.build_trees(inp.lp, inp.tok, inp.wl.budget)
@@ -394,21 +415,34 @@ def cpu_baseline(inp, depth, budget_s=15.0):
     rng = np.random.default_rng(12345)
     order = rng.permutation(B * T * H).astype(np.int32)
     done_rows, flops, t_used = 0, 0.0, 0.0
+    d_out = d_lse = 0.0
     chunk = 32
     while t_used < budget_s and done_rows < order.size:
         rows = order[done_rows:done_rows + chunk]
         t0 = time.perf_counter()
-        oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe, inp.page_table,
-                              inp.kv_len, mask, scale=synth.SCALE, dtype=inp.wl.dtype, rows=rows)
+        ref_out, ref_lse = oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe,
+                                                 inp.page_table, inp.kv_len, mask,
+                                                 scale=synth.SCALE, dtype=inp.wl.dtype, rows=rows)
         t_used += time.perf_counter() - t0
+        if gpu_out is not None:
+            live = np.isfinite(ref_lse)
+            d_out = max(d_out, float(np.abs(gpu_out[rows] - ref_out).max()))
+            if live.any():
+                d_lse = max(d_lse, float(np.abs(gpu_lse[rows][live] - ref_lse[live]).max()))
         b = rows // (T * H)
         t = (rows // H) % T
         d = trees["depth"][b, t]
         flops += float(((inp.prefix[b].astype(np.int64) + d + 1) * (d >= 0)).sum()) * FLOP_PER_KEY
         done_rows += rows.size
-    return {"value": round(flops / t_used / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{done_rows} seeded (b,t,h) rows of {B * T * H}, {t_used:.1f} s, fp64 C++"}
+    cores, model = host_cpu()
+    res = {"value": round(flops / t_used / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+           "kind": "oracle",
+           "sample": (f"{done_rows} seeded (b,t,h) rows of {B * T * H}, {t_used:.1f} s, fp64 C++"
+                      + (", extrapolated per flop" if done_rows < B * T * H else ", every row")),
+           "host": f"{cores} logical cores, {model}"}
+    if gpu_out is not None:
+        res["parity_on_sample"] = {"rows": done_rows, "out_max_abs": d_out, "lse_max_abs": d_lse}
+    return res
 
 
 def run_reference(args):
@@ -438,7 +472,7 @@ def run_reference(args):
         "data": "synthetic (seeded; no dataset or weights)", "impl": "reference",
         "config": cfg,
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": vals[0]["sample"]},
+                         "sample": vals[0]["sample"], "host": vals[0]["host"]},
         "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
