@@ -45,7 +45,7 @@ def _load():
         lib.or_build_tree.restype = i32
         lib.or_ancestor_mask.argtypes = [P, i32, i32, P, P]
         lib.or_ancestor_mask.restype = None
-        lib.or_attention_rows.argtypes = [i32, i32, i32, i32, i32, f64, i32,
+        lib.or_attention_rows.argtypes = [i32, i32, i32, i32, i32, f64, i32, i32, f64,
                                           P, P, P, P, i32, P, i32, P, P, P, P,
                                           i32, P, P, P]
         lib.or_attention_rows.restype = None
@@ -53,6 +53,8 @@ def _load():
         lib.or_merge.restype = None
         lib.or_tree_accept.argtypes = [P, P, P, i32, i32, P, P, P]
         lib.or_tree_accept.restype = None
+        lib.or_decode_e4m3.argtypes = [P, i64, P]
+        lib.or_decode_e4m3.restype = None
         _lib = lib
     return _lib
 
@@ -98,21 +100,38 @@ def ancestor_mask(parents: np.ndarray):
     return mask, status
 
 
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """FP8 E4M3 codes (uint8) -> float64 values (NaN for the two NaN codes)."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, np.uint8)
+    out = np.empty(codes.shape, np.float64)
+    lib.or_decode_e4m3(_ptr(codes), codes.size, _ptr(out))
+    return out
+
+
+_DTYPES = {"f32": (0, np.float32), "bf16": (1, np.uint16), "fp8_e4m3": (2, np.uint8)}
+
+
 def attention_rows(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, *, scale: float,
                    dtype: str, rows: Optional[np.ndarray] = None, key_lo=None, key_hi=None,
-                   page_size: int = 64):
+                   page_size: int = 64, kv_dtype: Optional[str] = None, kv_scale: float = 1.0):
     """Masked attention for flat rows (b*T + t)*H + h (all rows if ``rows`` is None).
 
-    q_nope [B,T,H,Dc], q_pe [B,T,H,Dr], c_kv [pages,page,Dc], k_pe [pages,page,Dr]
-    as float32 arrays (dtype "f32") or uint16 bf16 bit patterns (dtype "bf16").
+    q_nope [B,T,H,Dc], q_pe [B,T,H,Dr] as float32 arrays (dtype "f32") or uint16
+    bf16 bit patterns (dtype "bf16"); c_kv [pages,page,Dc], k_pe [pages,page,Dr]
+    in kv_dtype (default: dtype; "fp8_e4m3" = uint8 FP8 E4M3 codes), each cached
+    element standing for kv_scale times its stored value.
     Returns (out [n, Dc] float64, lse [n] float64).
     """
     lib = _load()
     B, T, H, Dc = q_nope.shape
     Dr = q_pe.shape[-1]
-    dt = {"f32": 0, "bf16": 1}[dtype]
-    want = np.float32 if dt == 0 else np.uint16
-    arrs = [np.ascontiguousarray(a, want) for a in (q_nope, q_pe, c_kv, k_pe)]
+    dt, want = _DTYPES[dtype]
+    if dt == 2:
+        raise ValueError("queries are f32 or bf16")
+    kdt, kwant = _DTYPES[kv_dtype or dtype]
+    arrs = [np.ascontiguousarray(a, want) for a in (q_nope, q_pe)]
+    arrs += [np.ascontiguousarray(a, kwant) for a in (c_kv, k_pe)]
     page_table = np.ascontiguousarray(page_table, np.int32)
     kv_len = np.ascontiguousarray(kv_len, np.int32)
     mask = np.ascontiguousarray(mask, np.uint64)
@@ -125,7 +144,8 @@ def attention_rows(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, *, scale:
     hi = None if key_hi is None else np.ascontiguousarray(key_hi, np.int32)
     out = np.zeros((n, Dc), np.float64)
     lse = np.zeros(n, np.float64)
-    lib.or_attention_rows(B, T, H, Dc, Dr, float(scale), dt, *[_ptr(a) for a in arrs],
+    lib.or_attention_rows(B, T, H, Dc, Dr, float(scale), dt, kdt, float(kv_scale),
+                          *[_ptr(a) for a in arrs],
                           page_size, _ptr(page_table), page_table.shape[1], _ptr(kv_len),
                           _ptr(mask), _ptr(lo), _ptr(hi), n, _ptr(rows), _ptr(out), _ptr(lse))
     return out, lse

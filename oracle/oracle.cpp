@@ -23,7 +23,9 @@
 // Pins (tests/): brute-force softmax on tiny inputs, hand-worked 3-node
 // trees, chain tree == causal attention, popcount(mask) == depth + 1,
 // page-table permutation invariance, split+merge == unsplit, brute-force
-// enumeration of the best-first tree on tiny (k, L).
+// enumeration of the best-first tree on tiny (k, L); the FP8 E4M3 decoder
+// against the format's closed-form values and against torch's float8_e4m3fn
+// conversion of all 256 codes.
 
 #include <cmath>
 #include <cstdint>
@@ -35,10 +37,27 @@ namespace {
 
 constexpr double kNegInf = -std::numeric_limits<double>::infinity();
 
-// Element fetch: dtype 0 = float32 storage, 1 = bf16 bit patterns.  Both
-// widen to double exactly.
+// One FP8 E4M3 code as a double, from the OCP 8-bit floating point format
+// definition (OFP8, the E4M3 encoding): bit 7 sign, bits 6..3 exponent field
+// E with bias 7, bits 2..0 mantissa M.  E = 0 is subnormal, M/8 * 2^-6; the
+// other fields are normal, (1 + M/8) * 2^(E - 7); the one pattern E = 15,
+// M = 7 is NaN (the format has no infinities, so its largest value is
+// 1.75 * 2^8 = 448).  Every code widens to double exactly.
+double decode_e4m3(uint8_t code) {
+  const int sign = code >> 7;
+  const int e = (code >> 3) & 15;
+  const int m = code & 7;
+  if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+  const double mag = e == 0 ? std::ldexp(static_cast<double>(m) / 8.0, -6)
+                            : std::ldexp(1.0 + static_cast<double>(m) / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+// Element fetch: dtype 0 = float32 storage, 1 = bf16 bit patterns, 2 = FP8
+// E4M3 codes.  All widen to double exactly.
 inline double fetch(const void* base, int64_t idx, int dtype) {
   if (dtype == 0) return static_cast<double>(static_cast<const float*>(base)[idx]);
+  if (dtype == 2) return decode_e4m3(static_cast<const uint8_t*>(base)[idx]);
   uint32_t bits = static_cast<uint32_t>(static_cast<const uint16_t*>(base)[idx]) << 16;
   float f;
   std::memcpy(&f, &bits, sizeof f);
@@ -64,6 +83,11 @@ bool better(const Cand& a, const Cand& b) {
 }  // namespace
 
 extern "C" {
+
+// FP8 E4M3 codes -> doubles (decode_e4m3 above), for the format's pins.
+void or_decode_e4m3(const uint8_t* codes, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = decode_e4m3(codes[i]);
+}
 
 // Best-first draft-tree builder ([MC] "The Context", item 1; [SP] "Why This
 // Message Was Written").  lp/tok are [L][K]: row d holds the drafter's top-K
@@ -151,9 +175,13 @@ void or_ancestor_mask(const int32_t* parents, int B, int T, uint64_t* mask,
 //   m = max s_j,  l = sum exp(s_j - m)
 //   out = sum_j exp(s_j - m) / l * c_kv_j,   lse = m + ln l
 // No visible key, or the row's own tree bit clear: out = 0, lse = -inf.
-// dtype: 0 = float32 inputs, 1 = bf16 bit patterns.  Outputs are float64.
+// dtype (queries): 0 = float32 inputs, 1 = bf16 bit patterns.  kv_dtype
+// (c_kv, k_pe): the same codes, or 2 = FP8 E4M3 codes; a cached element is
+// kv_scale times its stored value (the latent cache kept at 8 bits with one
+// scale for the whole tensor; not a step the pages describe).  Every c_kv_j
+// and k_pe_j above is that scaled value.  Outputs are float64.
 void or_attention_rows(int B, int T, int H, int Dc, int Dr, double scale, int dtype,
-                       const void* q_nope, const void* q_pe, const void* c_kv,
+                       int kv_dtype, double kv_scale, const void* q_nope, const void* q_pe, const void* c_kv,
                        const void* k_pe, int page_size, const int32_t* page_table,
                        int max_pages, const int32_t* kv_len, const uint64_t* mask,
                        const int32_t* key_lo, const int32_t* key_hi,
@@ -188,9 +216,9 @@ void or_attention_rows(int B, int T, int H, int Dc, int Dr, double scale, int dt
       const int64_t kr = page * page_size + j % page_size;
       double dot = 0.0;
       for (int d = 0; d < Dc; ++d)
-        dot += fetch(q_nope, r * Dc + d, dtype) * fetch(c_kv, kr * Dc + d, dtype);
+        dot += fetch(q_nope, r * Dc + d, dtype) * (kv_scale * fetch(c_kv, kr * Dc + d, kv_dtype));
       for (int e = 0; e < Dr; ++e)
-        dot += fetch(q_pe, r * Dr + e, dtype) * fetch(k_pe, kr * Dr + e, dtype);
+        dot += fetch(q_pe, r * Dr + e, dtype) * (kv_scale * fetch(k_pe, kr * Dr + e, kv_dtype));
       s.push_back(scale * dot);
       krow.push_back(kr);
     }
@@ -201,7 +229,7 @@ void or_attention_rows(int B, int T, int H, int Dc, int Dr, double scale, int dt
     for (double v : s) l += std::exp(v - m);
     for (size_t k = 0; k < s.size(); ++k) {
       const double w = std::exp(s[k] - m) / l;
-      for (int d = 0; d < Dc; ++d) o[d] += w * fetch(c_kv, krow[k] * Dc + d, dtype);
+      for (int d = 0; d < Dc; ++d) o[d] += w * (kv_scale * fetch(c_kv, krow[k] * Dc + d, kv_dtype));
     }
     lse[ri] = m + std::log(l);
   }

@@ -19,7 +19,10 @@ Draw order for one workload (one numpy PCG64 stream, seed 0xDD7EE000 + i):
   2. ragged prefix lengths,
   3. the page permutation,
   4. q_nope, q_pe, c_kv, k_pe (N(0,1); rounded to bf16 by
-     round-to-nearest-even for bf16 workloads).
+     round-to-nearest-even for bf16 workloads).  Workloads whose latent cache
+     is kept as FP8 E4M3 codes draw c_kv and k_pe as codes instead (see
+     ``draw_e4m3_codes``); the cache then stands for kv_scale times the coded
+     values.
 """
 from __future__ import annotations
 
@@ -53,6 +56,8 @@ class Workload:
     paged: bool = True            # shuffled 64-token pages (else identity table)
     splits: int = 1               # split-KV chunks for the flash-decode path (0: the library plans)
     seed_index: int = 0
+    kv: str = "same"              # latent cache storage: "same" as dtype, or "fp8_e4m3" codes
+    kv_scale: float = 1.0         # value of one cache unit (FP8 cache only)
 
     @property
     def T(self) -> int:
@@ -74,6 +79,14 @@ WORKLOADS = {
                                 budget=32, topk=8, paged=True, seed_index=3),
     "bf16-long-prefix": Workload("bf16-long-prefix", "bf16", B=4, H=64, P=131072,
                                  budget=64, topk=8, paged=True, splits=16, seed_index=4),
+    # FP8 latent cache (one scale per tensor) under the fp32 and bf16 query
+    # shapes above; 7/16 is not a power of two, so scaling is not exact.
+    "fp32-fp8kv": Workload("fp32-fp8kv", "f32", B=1, H=64, P=2048, budget=32, topk=8,
+                           paged=True, splits=0, seed_index=5, kv="fp8_e4m3",
+                           kv_scale=0.4375),
+    "bf16-fp8kv-deep": Workload("bf16-fp8kv-deep", "bf16", B=16, H=64, P=4096, budget=64,
+                                topk=2, paged=True, seed_index=6, kv="fp8_e4m3",
+                                kv_scale=0.4375),
 }
 WORKLOAD_ORDER = ["fp32-tiny", "fp32-page-test", "bf16-deep", "bf16-b64-ragged",
                   "bf16-long-prefix"]
@@ -94,6 +107,19 @@ def bf16_to_f32(u: np.ndarray) -> np.ndarray:
     return (u.astype(np.uint32) << 16).view(np.float32)
 
 
+def draw_e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Random FP8 E4M3 codes (uint8), drawn field by field: a fair sign bit, an
+    exponent field 7 + round(N(0, 1)) clipped to [0, 15] (so magnitudes sit
+    around 1 and reach the subnormal and largest binades now and then) and a
+    uniform 3-bit mantissa.  The NaN pattern (exponent 15, mantissa 7) is
+    replaced by mantissa 6, the largest finite magnitude."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8)
+    exp = np.clip(np.rint(7.0 + rng.standard_normal(size=shape)), 0, 15).astype(np.uint8)
+    man = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    man = np.where((exp == 15) & (man == 7), np.uint8(6), man).astype(np.uint8)
+    return ((sign << 7) | (exp << 3) | man).astype(np.uint8)
+
+
 def drafter_topk(rng: np.random.Generator, L: int, K: int, vocab: int = VOCAB,
                  sigma: float = 2.0) -> Tuple[np.ndarray, np.ndarray]:
     """Synthetic drafter output: per-depth top-K log-probs (descending) and token ids.
@@ -112,7 +138,8 @@ def drafter_topk(rng: np.random.Generator, L: int, K: int, vocab: int = VOCAB,
 
 @dataclasses.dataclass
 class Inputs:
-    """Host arrays of one workload.  Values of bf16 workloads are uint16 bit patterns."""
+    """Host arrays of one workload.  Values of bf16 workloads are uint16 bit patterns;
+    an FP8 cache holds uint8 E4M3 codes."""
 
     wl: Workload
     lp: np.ndarray          # [B, L, K] float64 drafter log-probs
@@ -184,8 +211,12 @@ def make_inputs(wl: Workload, *, B: Optional[int] = None, H: Optional[int] = Non
     if with_tensors:
         q_nope = draw((Bn, T, Hn, D_LATENT))
         q_pe = draw((Bn, T, Hn, D_ROPE))
-        c_kv = draw((num_pages, PAGE_SIZE, D_LATENT))
-        k_pe = draw((num_pages, PAGE_SIZE, D_ROPE))
+        if wl.kv == "fp8_e4m3":
+            c_kv = draw_e4m3_codes(rng, (num_pages, PAGE_SIZE, D_LATENT))
+            k_pe = draw_e4m3_codes(rng, (num_pages, PAGE_SIZE, D_ROPE))
+        else:
+            c_kv = draw((num_pages, PAGE_SIZE, D_LATENT))
+            k_pe = draw((num_pages, PAGE_SIZE, D_ROPE))
     else:
         q_nope = q_pe = c_kv = k_pe = None
     return Inputs(wl, lp, tok, prefix, kv_len, page_table, num_pages,

@@ -31,8 +31,13 @@ def to_device(inp: synth.Inputs, parents: np.ndarray, device="cuda"):
             t = t.view(torch.int16).view(torch.bfloat16)
         return t.to(device)
 
+    def cache(a):
+        if inp.wl.kv == "fp8_e4m3":
+            return torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e4m3fn).to(device)
+        return vals(a)
+
     return dict(
-        q_nope=vals(inp.q_nope), q_pe=vals(inp.q_pe), c_kv=vals(inp.c_kv), k_pe=vals(inp.k_pe),
+        q_nope=vals(inp.q_nope), q_pe=vals(inp.q_pe), c_kv=cache(inp.c_kv), k_pe=cache(inp.k_pe),
         page_table=torch.from_numpy(inp.page_table).to(device),
         kv_len=torch.from_numpy(inp.kv_len).to(device),
         parents=torch.from_numpy(np.ascontiguousarray(parents, np.int32)).to(device),
@@ -42,7 +47,14 @@ def to_device(inp: synth.Inputs, parents: np.ndarray, device="cuda"):
 def oracle_rows(inp: synth.Inputs, mask: np.ndarray, rows=None, key_lo=None, key_hi=None):
     return oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe, inp.page_table,
                                  inp.kv_len, mask, scale=synth.SCALE, dtype=inp.wl.dtype,
-                                 rows=rows, key_lo=key_lo, key_hi=key_hi)
+                                 rows=rows, key_lo=key_lo, key_hi=key_hi, **kv_kwargs(inp))
+
+
+def kv_kwargs(inp: synth.Inputs) -> dict:
+    """Cache storage arguments of the oracle for this workload."""
+    if inp.wl.kv == "fp8_e4m3":
+        return dict(kv_dtype="fp8_e4m3", kv_scale=inp.wl.kv_scale)
+    return {}
 
 
 def compare(out_gpu, lse_gpu, out_ref, lse_ref, dtype: str, what: str = ""):

@@ -461,3 +461,80 @@ def test_tree_accept_bruteforce(seed):
         chain, nt = accept_bruteforce(list(par[b]), list(tok[b]), list(target[b]))
         assert path[b, :alen[b]].tolist() == chain and nxt[b] == nt
         assert alen[b] == len(chain) and (path[b, alen[b]:] == -1).all()
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 latent cache
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decoder_closed_forms():
+    g = json.load(open(os.path.join(GOLDEN, "e4m3_codes.json")))
+    codes = np.array([int(c["code"], 16) for c in g["codes"]], np.uint8)
+    got = oracle.decode_e4m3(codes)
+    for c, v in zip(g["codes"], got):
+        want = math.ldexp(c["num"], c["exp2"])
+        assert v == want and math.copysign(1.0, v) == math.copysign(1.0, want), c
+    nans = oracle.decode_e4m3(np.array([int(c, 16) for c in g["nan_codes"]], np.uint8))
+    assert np.isnan(nans).all()
+
+
+def test_e4m3_decoder_matches_torch_on_all_codes():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.decode_e4m3(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def fp8_case(seed, B=2, T=6, H=3, P=(0, 70)):
+    """small_inputs with the cache replaced by E4M3 codes (all finite codes used)."""
+    d = small_inputs(seed, B=B, T=T, H=H, P=P)
+    rng = np.random.default_rng(seed + 100)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    d["c_kv"] = rng.choice(finite, size=d["c_kv"].shape).astype(np.uint8)
+    d["k_pe"] = rng.choice(finite, size=d["k_pe"].shape).astype(np.uint8)
+    return d
+
+
+@pytest.mark.parametrize("seed,kv_scale", [(4, 0.4375), (5, 1.0 / 448.0), (6, 3.0)])
+def test_fp8_cache_matches_dense_bruteforce(seed, kv_scale):
+    """The oracle on codes == the numpy brute force on torch-decoded, scaled values."""
+    import torch
+    d = fp8_case(seed)
+    dec = lambda a: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mask, status = oracle.ancestor_mask(d["parents"])
+    out, lse = oracle.attention_rows(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"],
+                                     d["page_table"], d["kv_len"], mask, scale=synth.SCALE,
+                                     dtype="f32", kv_dtype="fp8_e4m3", kv_scale=kv_scale)
+    ref_out, ref_lse = dense_reference(d["q_nope"], d["q_pe"], kv_scale * dec(d["c_kv"]),
+                                       kv_scale * dec(d["k_pe"]), d["page_table"], d["kv_len"],
+                                       d["parents"], synth.SCALE)
+    live = np.isfinite(ref_lse.reshape(-1))
+    assert live.any()
+    np.testing.assert_allclose(out, ref_out.reshape(out.shape), rtol=1e-12,
+                               atol=1e-12 * max(1.0, 448 * kv_scale))
+    np.testing.assert_allclose(lse[live], ref_lse.reshape(-1)[live], rtol=1e-12, atol=1e-9)
+
+
+def test_fp8_cache_identical_keys_closed_form():
+    """Every visible key the same code c: out = kv_scale * value(c), lse = s + ln(count)."""
+    T, H, P, kv_scale = 4, 2, 10, 0.4375
+    d = small_inputs(21, B=1, T=T, H=H, P=P, parents=[[-1, 0, 1, 1]])
+    d["c_kv"] = np.full(d["c_kv"].shape, 0x3F, np.uint8)     # 1.875
+    d["k_pe"] = np.full(d["k_pe"].shape, 0xC0, np.uint8)     # -2
+    mask, _ = oracle.ancestor_mask(d["parents"])
+    out, lse = oracle.attention_rows(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"],
+                                     d["page_table"], d["kv_len"], mask, scale=synth.SCALE,
+                                     dtype="f32", kv_dtype="fp8_e4m3", kv_scale=kv_scale)
+    depth = [0, 1, 2, 2]
+    for t in range(T):
+        for h in range(H):
+            r = t * H + h
+            q = d["q_nope"][0, t, h].astype(np.float64)
+            qp = d["q_pe"][0, t, h].astype(np.float64)
+            s = synth.SCALE * kv_scale * (1.875 * q.sum() - 2.0 * qp.sum())
+            np.testing.assert_allclose(out[r], np.full(DC, kv_scale * 1.875), rtol=1e-14)
+            assert abs(lse[r] - (s + math.log(P + depth[t] + 1))) < 1e-10
