@@ -73,10 +73,11 @@ def work(inp, depth):
     """Algorithmic flops and bytes of one step (visible keys only)."""
     B, T, H = inp.wl.B, inp.T, inp.wl.H
     e = 2 if inp.wl.dtype == "bf16" else 4
+    ekv = 1 if inp.wl.kv == "fp8_e4m3" else e
     present = depth >= 0                                    # [B, T]
     vis = (inp.prefix[:, None].astype(np.int64) + depth + 1) * present
     flops = float(vis.sum()) * H * FLOP_PER_KEY
-    kv_bytes = float(inp.kv_len.astype(np.int64).sum()) * (synth.D_LATENT + synth.D_ROPE) * e
+    kv_bytes = float(inp.kv_len.astype(np.int64).sum()) * (synth.D_LATENT + synth.D_ROPE) * ekv
     q_bytes = float(B * T * H) * (synth.D_LATENT + synth.D_ROPE) * e
     out_bytes = float(B * T * H) * (synth.D_LATENT * e + 4)
     return flops, kv_bytes + q_bytes + out_bytes
@@ -181,7 +182,8 @@ def config_of(wl, S, world, flops, alg_bytes):
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T,
             "prefix": list(wl.P) if isinstance(wl.P, tuple) else wl.P,
             "tree": f"best-first top-{wl.topk}, depth<={wl.max_depth}, budget {wl.budget}",
-            "kv": "64-token pages, shuffled" if wl.paged else "contiguous",
+            "kv": ("64-token pages, shuffled" if wl.paged else "contiguous")
+                  + (f", FP8 E4M3 cache x {wl.kv_scale}" if wl.kv == "fp8_e4m3" else ""),
             "num_splits": S, "parallelism": f"replicas x{world} (independent requests)",
             "l2": ("inputs larger than the 126 MB L2, no flush" if alg_bytes > 126e6 else
                    "inputs fit in the 126 MB L2 and are not flushed (warm-cache figure)"),
@@ -198,6 +200,8 @@ def run_gpu(args):
     inp = synth.make_inputs(wl, seed=rank_seed(wl, rank))
     dev = torch.device("cuda", local)
     bf16 = wl.dtype == "bf16"
+    fp8 = wl.kv == "fp8_e4m3"
+    tc = bf16 and not fp8        # the tensor-core kernel; everything else runs on CUDA cores
     tdt = torch.bfloat16 if bf16 else torch.float32
 
     def to_dev(a):
@@ -207,7 +211,10 @@ def run_gpu(args):
         return t.to(dev)
 
     q_nope, q_pe = to_dev(inp.q_nope), to_dev(inp.q_pe)
-    c_kv, k_pe = to_dev(inp.c_kv), to_dev(inp.k_pe)
+    if fp8:
+        c_kv, k_pe = (torch.from_numpy(a).view(torch.float8_e4m3fn).to(dev) for a in (inp.c_kv, inp.k_pe))
+    else:
+        c_kv, k_pe = to_dev(inp.c_kv), to_dev(inp.k_pe)
     page_table = torch.from_numpy(inp.page_table).to(dev)
     kv_len = torch.from_numpy(inp.kv_len).to(dev)
     # draft trees from the library's GPU best-first builder
@@ -222,7 +229,7 @@ def run_gpu(args):
     tstat = torch.empty(B, device=dev, dtype=torch.int32)
     splits = args.splits if args.splits is not None else wl.splits
     vargs = va.make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, out, lse,
-                         scale=synth.SCALE, num_splits=splits)
+                         scale=synth.SCALE, num_splits=splits, kv_scale=wl.kv_scale)
     S = va.num_splits(vargs)
     wbytes = va.workspace_bytes(vargs)
     ws = torch.empty(max(wbytes, 256), device=dev, dtype=torch.uint8) if wbytes else None
@@ -298,7 +305,8 @@ def run_gpu(args):
         st_["ws"] = torch.empty(max(wbytes, 256), device=dev, dtype=torch.uint8) if wbytes else None
         st_["args"] = va.make_args(st_["q_nope"], st_["q_pe"], c_kv, k_pe, st_["page_table"],
                                    st_["kv_len"], st_["mask"], st_["out"], st_["lse"],
-                                   scale=synth.SCALE, num_splits=splits, workspace=st_["ws"])
+                                   scale=synth.SCALE, num_splits=splits, workspace=st_["ws"],
+                                   kv_scale=wl.kv_scale)
         sets.append(st_)
     s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "run", "out")}
@@ -349,10 +357,10 @@ def run_gpu(args):
     e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
 
     hbm, tc_peak, tc_sust, peak_src = peaks()
-    kernel_src = "speculative_decoding_tree_va_b200/csrc/" + ("va_attn_tc.cu" if bf16 else "va_attn_simt.cu")
+    kernel_src = "speculative_decoding_tree_va_b200/csrc/" + ("va_attn_tc.cu" if tc else "va_attn_simt.cu")
     traffic = recorded_traffic(kernel_src, wl.name) if S == 1 else None
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    roof_us = max(flops / ((tc_peak if bf16 else FP32_FFMA_PEAK) * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
+    roof_us = max(flops / ((tc_peak if tc else FP32_FFMA_PEAK) * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
     clocks = clk.summary()
     if dist is not None:
         dist.destroy_process_group()
@@ -368,15 +376,15 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "us_per_step": round(ms_step * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded; no dataset or weights)",
+        "dtype": "bf16" if tc else "f32", "data": "synthetic (seeded; no dataset or weights)",
         "config": config_of(wl, S, world, flops, alg_bytes),
-        "roofline": {"bound": "tensor" if bf16 else "alu", "achieved": round(achieved, 2),
-                     "peak": tc_peak if bf16 else FP32_FFMA_PEAK,
-                     "unit": "TFLOP/s", "frac": round(achieved / (tc_peak if bf16 else FP32_FFMA_PEAK), 4),
+        "roofline": {"bound": "tensor" if tc else "alu", "achieved": round(achieved, 2),
+                     "peak": tc_peak if tc else FP32_FFMA_PEAK,
+                     "unit": "TFLOP/s", "frac": round(achieved / (tc_peak if tc else FP32_FFMA_PEAK), 4),
                      "traffic": traffic,
-                     "peak_source": (f"{peak_src} bf16 dense (burst); sustained {tc_sust}" if bf16 else
+                     "peak_source": (f"{peak_src} bf16 dense (burst); sustained {tc_sust}" if tc else
                                      "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz"),
-                     "kernel": "attn_tc_kernel" if bf16 else "attn_simt_kernel",
+                     "kernel": "attn_tc_kernel" if tc else "attn_simt_kernel",
                      "kernel_us": round(attn_ms * 1e3, 1), "roofline_us": round(roof_us, 1),
                      "frac_of_step_roofline": round(roof_us / (ms_step * 1e3), 4)},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
@@ -416,13 +424,16 @@ def cpu_baseline(inp, depth, budget_s=15.0, gpu_out=None, gpu_lse=None):
     order = rng.permutation(B * T * H).astype(np.int32)
     done_rows, flops, t_used = 0, 0.0, 0.0
     d_out = d_lse = 0.0
+    kv_args = (dict(kv_dtype="fp8_e4m3", kv_scale=inp.wl.kv_scale) if inp.wl.kv == "fp8_e4m3"
+               else {})
     chunk = 32
     while t_used < budget_s and done_rows < order.size:
         rows = order[done_rows:done_rows + chunk]
         t0 = time.perf_counter()
         ref_out, ref_lse = oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe,
                                                  inp.page_table, inp.kv_len, mask,
-                                                 scale=synth.SCALE, dtype=inp.wl.dtype, rows=rows)
+                                                 scale=synth.SCALE, dtype=inp.wl.dtype, rows=rows,
+                                                 **kv_args)
         t_used += time.perf_counter() - t0
         if gpu_out is not None:
             live = np.isfinite(ref_lse)

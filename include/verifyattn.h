@@ -163,6 +163,8 @@ typedef struct va_attn_args {
   void* workspace;    /* [device] split-KV partials, >= va_workspace_bytes()    */
   size_t workspace_bytes;
   int flags;          /* VA_FLAG_* below                                        */
+  float kv_scale;     /* with VA_FLAG_KV_FP8_E4M3: the value of one cache unit
+                         (finite, > 0); ignored otherwise                      */
 } va_attn_args;
 
 /* Run bf16 inputs on the CUDA-core FFMA kernel instead of the tensor-core
@@ -176,6 +178,19 @@ typedef struct va_attn_args {
  * -inf, va_device_timeouts() grows, and the context stays usable.  No copy
  * is in flight when the CTAs give up, so nothing lands after they exit. */
 #define VA_FLAG_TEST_STALL_MMA 2
+
+/* Latent cache kept as FP8 E4M3 codes, one byte per element, with one scale
+ * for the whole cache: c_kv is uint8 [num_pages, 64, 512], k_pe uint8
+ * [num_pages, 64, 64], and code x stands for kv_scale * value(x) in every
+ * formula of va_verify_attn.  E4M3 is the OCP 8-bit floating point format
+ * (sign, 4-bit exponent with bias 7, 3-bit mantissa; exponent field 0 is
+ * subnormal; S.1111.111 is NaN; no infinities; largest magnitude 448).  The
+ * cache takes half the bytes of a bf16 one; queries and outputs keep `dtype`
+ * (fp32 or bf16).  The pages keep the cache in the model's dtype: this is an
+ * addition.  Both query types run on the CUDA-core kernel, which widens every
+ * code exactly.  kv_scale must be finite and > 0, else VA_ERR_INVALID_ARG;
+ * VA_FLAG_TEST_STALL_MMA is rejected with this flag. */
+#define VA_FLAG_KV_FP8_E4M3 4
 
 /*
  * Workspace needed by va_verify_attn for these arguments (0 for a single
@@ -204,7 +219,8 @@ int va_num_splits(const va_attn_args* args);
  * With S > 1 splits, split s covers keys [s*C, min((s+1)*C, kv_len)) with
  * C = ceil(ceil(kv_len / S) / 256) * 256; the partials go to the workspace
  * and va_merge combines them on the same stream.
- * bf16 runs on tensor cores with fp32 accumulation; fp32 on CUDA cores.
+ * bf16 runs on tensor cores with fp32 accumulation; fp32, and any call with
+ * an FP8 cache (VA_FLAG_KV_FP8_E4M3), on CUDA cores.
  * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, B >= 0.  Slots past
  * kv_len in a request's last page may hold any finite values (they are
  * multiplied by exact zeros; NaN or Inf there would propagate).

@@ -22,6 +22,7 @@ VA_OK, VA_ERR_INVALID_ARG, VA_ERR_UNSUPPORTED, VA_ERR_CUDA, VA_ERR_INVALID_TREE 
 VA_F32, VA_BF16 = 0, 1
 VA_FLAG_BF16_CUDA_CORES = 1
 VA_FLAG_TEST_STALL_MMA = 2  # test hook: the tensor-core kernel's bounded waits expire
+VA_FLAG_KV_FP8_E4M3 = 4     # latent cache as FP8 E4M3 codes times kv_scale
 D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",
@@ -44,6 +45,7 @@ class VaAttnArgs(ctypes.Structure):
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("req_status", ctypes.c_void_p),
         ("num_splits", ctypes.c_int), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("flags", ctypes.c_int),
+        ("kv_scale", ctypes.c_float),
     ]
 
 
@@ -155,9 +157,18 @@ def build_tree_mask(parents, stream=None):
     return mask, status
 
 
+def _fp8_cache(c_kv) -> bool:
+    import torch
+    return c_kv.dtype in (torch.uint8, torch.float8_e4m3fn)
+
+
 def make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, out, lse, *, scale: float,
-              num_splits: int = 0, workspace=None, req_status=None, flags: int = 0) -> VaAttnArgs:
-    """Fill a VaAttnArgs from torch tensors (no checks beyond what the library does)."""
+              num_splits: int = 0, workspace=None, req_status=None, flags: int = 0,
+              kv_scale: float = 1.0) -> VaAttnArgs:
+    """Fill a VaAttnArgs from torch tensors (no checks beyond what the library does).
+
+    A uint8 or float8_e4m3fn cache (c_kv, k_pe) sets VA_FLAG_KV_FP8_E4M3 with
+    kv_scale, the value of one cache unit."""
     import torch
     B, T, H, _ = q_nope.shape
     dt = {torch.float32: VA_F32, torch.bfloat16: VA_BF16}[q_nope.dtype]
@@ -173,6 +184,9 @@ def make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, out, lse,
     a.workspace = None if workspace is None else workspace.data_ptr()
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.flags = flags
+    if _fp8_cache(c_kv):
+        a.flags |= VA_FLAG_KV_FP8_E4M3
+        a.kv_scale = float(kv_scale)
     return a
 
 
@@ -190,12 +204,14 @@ def verify_attn_args(args: VaAttnArgs, stream=None):
 
 def verify_attn(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, *, scale: float,
                 num_splits: int = 0, out=None, lse=None, workspace=None, req_status=None,
-                flags: int = 0, stream=None):
+                flags: int = 0, kv_scale: float = 1.0, stream=None):
     """Tree-verify MLA-absorb attention.  Allocates out/lse/workspace when not given.
 
-    q_nope [B,T,H,512], q_pe [B,T,H,64], c_kv [pages,64,512], k_pe [pages,64,64]
-    (float32 or bfloat16, cuda), page_table int32 [B, max_pages], kv_len int32 [B],
-    tree_mask int64 [B,T,W] from build_tree_mask.  Returns (out, lse)."""
+    q_nope [B,T,H,512], q_pe [B,T,H,64] (float32 or bfloat16, cuda); c_kv
+    [pages,64,512], k_pe [pages,64,64] in the query dtype, or FP8 E4M3 codes
+    (uint8 / float8_e4m3fn) standing for kv_scale times their values;
+    page_table int32 [B, max_pages], kv_len int32 [B], tree_mask int64 [B,T,W]
+    from build_tree_mask.  Returns (out, lse) in the query dtype."""
     import torch
     B, T, H, _ = q_nope.shape
     if out is None:
@@ -204,7 +220,7 @@ def verify_attn(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, *, scal
         lse = torch.empty(B, T, H, device=q_nope.device, dtype=torch.float32)
     args = make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, tree_mask, out, lse,
                      scale=scale, num_splits=num_splits, workspace=workspace,
-                     req_status=req_status, flags=flags)
+                     req_status=req_status, flags=flags, kv_scale=kv_scale)
     need = workspace_bytes(args)
     if need and workspace is None:
         workspace = torch.empty(need, device=q_nope.device, dtype=torch.uint8)

@@ -1,6 +1,7 @@
 // C ABI of libverifyattn: argument checks, split planning, dispatch.
 // Every entry point validates on the host and returns a va_status before
 // launching anything; the caller owns all device memory.
+#include <cfloat>
 #include <cstdio>
 
 #include "va_common.cuh"
@@ -20,10 +21,12 @@ int check_args(const va_attn_args* a) {
   if (a->B < 0 || a->H < 1 || a->T < 1 || a->T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
   if (a->page_size != VA_PAGE_SIZE) return VA_ERR_UNSUPPORTED;
   if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
-  if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA)) return VA_ERR_INVALID_ARG;
-  if ((a->flags & VA_FLAG_TEST_STALL_MMA) &&
-      (a->dtype != VA_BF16 || (a->flags & VA_FLAG_BF16_CUDA_CORES)))
+  if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA | VA_FLAG_KV_FP8_E4M3))
+    return VA_ERR_INVALID_ARG;
+  if ((a->flags & VA_FLAG_TEST_STALL_MMA) && !va::uses_tensor_cores(*a))
     return VA_ERR_INVALID_ARG;  // only the tensor-core kernel has the hook
+  if ((a->flags & VA_FLAG_KV_FP8_E4M3) && !(a->kv_scale > 0.f && a->kv_scale <= FLT_MAX))
+    return VA_ERR_INVALID_ARG;  // NaN, zero, negative or infinite cache scale
   if (!(a->scale == a->scale)) return VA_ERR_INVALID_ARG;  // NaN scale
   if (a->B == 0) return VA_OK;
   if (a->num_pages < 1 || a->max_pages < 1) return VA_ERR_INVALID_ARG;
@@ -39,10 +42,6 @@ int check_args(const va_attn_args* a) {
   return VA_OK;
 }
 
-bool use_tensor_cores(const va_attn_args* a) {
-  return a->dtype == VA_BF16 && !(a->flags & VA_FLAG_BF16_CUDA_CORES);
-}
-
 // Split count: the caller's, or (num_splits == 0) the smallest power of two
 // that fills >= 90% of the last wave, keeping >= 1024 keys per split.  The
 // host does not see kv_len, so the planner uses the page-table capacity as
@@ -52,7 +51,7 @@ int plan_splits(const va_attn_args* a) {
   if (a->B == 0) return 1;
   const long long rows = (long long)a->T * a->H;
   long long units_per_split, slots;
-  if (use_tensor_cores(a)) {
+  if (va::uses_tensor_cores(*a)) {
     units_per_split = (long long)a->B * ((rows + 127) / 128);  // CTA pairs
     slots = kSms / 2;
   } else {
@@ -157,7 +156,7 @@ int va_verify_attn(const va_attn_args* args, va_stream_t stream) {
     lse_part = (float*)((char*)args->workspace + lse_off);
   }
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = use_tensor_cores(args) ? va::launch_attn_tc(*args, S, o_part, lse_part, s)
+  cudaError_t e = va::uses_tensor_cores(*args) ? va::launch_attn_tc(*args, S, o_part, lse_part, s)
                                          : va::launch_attn_simt(*args, S, o_part, lse_part, s);
   if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return VA_ERR_CUDA;

@@ -1,5 +1,6 @@
-// CUDA-core (FFMA) tree-verify attention: the fp32 path, and a second,
-// independent GPU path for bf16 inputs.
+// CUDA-core (FFMA) tree-verify attention: the fp32 path, a second,
+// independent GPU path for bf16 inputs, and the path for a latent cache kept
+// as FP8 E4M3 codes (either query type).
 //
 // Computes, per row (b, t, h), the masked softmax over the request's prefix
 // and the row's tree ancestors in the absorbed latent space (page "The
@@ -12,6 +13,12 @@
 // fp32 inputs) are shared by the 32 rows.  Scores: lane = key.  Output: lane
 // owns 16 of the 512 latent columns (4 groups of 4, 128 apart) for the
 // warp's 4 rows, so every row's softmax state lives in one warp.
+//
+// FP8 cache: codes are widened to fp32 while they are staged; the cache scale
+// is folded into the score scale and into the output normalisation, so the
+// inner loops are those of the other types.
+#include <cuda_fp8.h>
+
 #include "va_common.cuh"
 
 namespace va {
@@ -61,6 +68,21 @@ __device__ __forceinline__ void load_row_chunk(float* dst, const __nv_bfloat16* 
   reinterpret_cast<float4*>(dst)[1] = b;
 }
 
+// Load 16 FP8 E4M3 codes as fp32 into dst.  The hardware conversion to fp16
+// is exact for every finite code (E4M3 values are a subset of fp16's), and
+// so is fp16 -> fp32.  Code k of the 16 bytes lands in dst[k].
+__device__ __forceinline__ void load_row_chunk(float* dst, const uint8_t* src) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 lo(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3));
+    const __half2 hi(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3));
+    const float2 a = __half22float2(lo), b = __half22float2(hi);
+    reinterpret_cast<float4*>(dst)[i] = make_float4(a.x, a.y, b.x, b.y);
+  }
+}
+
 template <typename Tin>
 struct Elems {  // values per 16-byte chunk
   static constexpr int v = 16 / sizeof(Tin);
@@ -91,13 +113,17 @@ __device__ void stage_keys(float* sK, const Tin* __restrict__ c_kv, const Tin* _
   }
 }
 
-template <typename Tin, typename Tout>
+// Tq: query element type; Tkv: cache element type (Tq, or uint8_t E4M3
+// codes); Tout: output element type.  scale_log2 already holds the cache
+// scale; out_scale (the cache scale, 1 for an unscaled cache) multiplies the
+// normalised output.
+template <typename Tq, typename Tkv, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
-                 const Tin* __restrict__ c_kv, const Tin* __restrict__ k_pe, int num_pages,
+attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
+                 const Tkv* __restrict__ c_kv, const Tkv* __restrict__ k_pe, int num_pages,
                  const int32_t* __restrict__ page_table, int max_pages,
                  const int32_t* __restrict__ kv_len_arr, const uint64_t* __restrict__ tree_mask,
-                 int H, int T, float scale_log2, int S, Tout* __restrict__ out,
+                 int H, int T, float scale_log2, float out_scale, int S, Tout* __restrict__ out,
                  float* __restrict__ lse_out, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
@@ -124,7 +150,7 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
 
   // q rows -> shared (fp32).  Rows past R are zero.
   {
-    constexpr int V = Elems<Tin>::v;
+    constexpr int V = Elems<Tq>::v;
     constexpr int kChunksC = kDc / V, kChunks = kChunksC + kDr / V;
     for (int c = tid; c < kRows * kChunks; c += kThreads) {
       const int r = c / kChunks, part = c - r * kChunks;
@@ -132,7 +158,7 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
       const int row = row0 + r;
       if (row < R) {
         const size_t g = (size_t)b * R + row;
-        const Tin* src = part < kChunksC ? q_nope + g * kDc + part * V
+        const Tq* src = part < kChunksC ? q_nope + g * kDc + part * V
                                          : q_pe + g * kDr + (part - kChunksC) * V;
         load_row_chunk(dst, src);
       } else {
@@ -173,7 +199,7 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
     if (pg < 0 || pg >= num_pages) { bad_page = 1; return -1; }
     return pg;
   };
-  if (ntiles > 0) stage_keys<Tin>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
+  if (ntiles > 0) stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
   cp_async_commit();
 
   for (int it = 0; it < ntiles; ++it) {
@@ -182,7 +208,7 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
     __syncthreads();
     if (it + 1 < ntiles) {
       const int jn = lo + (it + 1) * kKeys;
-      stage_keys<Tin>((it & 1) ? sK0 : sK1, c_kv, k_pe, phys_of(jn), jn, hi, tid);
+      stage_keys<Tkv>((it & 1) ? sK0 : sK1, c_kv, k_pe, phys_of(jn), jn, hi, tid);
     }
     cp_async_commit();
 
@@ -259,7 +285,7 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
     const int row = row0 + warp * 4 + r;
     if (row >= R) continue;
     const bool empty = !(l[r] > 0.f) || !req_ok || bad_page;
-    const float inv = empty ? 0.f : 1.f / l[r];
+    const float inv = empty ? 0.f : out_scale / l[r];
     const float lse = empty ? -INFINITY : (m[r] + log2f(l[r])) * kLn2;
     const size_t g = (size_t)b * R + row;
     if (S == 1) {
@@ -282,20 +308,21 @@ attn_simt_kernel(const Tin* __restrict__ q_nope, const Tin* __restrict__ q_pe,
   }
 }
 
-template <typename Tin, typename Tout>
+template <typename Tq, typename Tkv, typename Tout>
 cudaError_t launch_typed(const va_attn_args& a, int S, float* o_part, float* lse_part,
                          cudaStream_t st) {
-  auto kern = attn_simt_kernel<Tin, Tout>;
+  auto kern = attn_simt_kernel<Tq, Tkv, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemTotal);
   if (e != cudaSuccess) return e;
   const int R = a.T * a.H;
   dim3 grid((R + kRows - 1) / kRows, a.B, S);
-  const float scale_log2 = a.scale * kLog2e;
+  const float kv_scale = (a.flags & VA_FLAG_KV_FP8_E4M3) ? a.kv_scale : 1.f;
+  const float scale_log2 = (a.scale * kv_scale) * kLog2e;
   kern<<<grid, kThreads, kSmemTotal, st>>>(
-      (const Tin*)a.q_nope, (const Tin*)a.q_pe, (const Tin*)a.c_kv, (const Tin*)a.k_pe,
-      a.num_pages, a.page_table, a.max_pages, a.kv_len, a.tree_mask, a.H, a.T, scale_log2, S,
-      (Tout*)a.out, a.lse, o_part, lse_part, a.req_status, a.B);
+      (const Tq*)a.q_nope, (const Tq*)a.q_pe, (const Tkv*)a.c_kv, (const Tkv*)a.k_pe,
+      a.num_pages, a.page_table, a.max_pages, a.kv_len, a.tree_mask, a.H, a.T, scale_log2,
+      kv_scale, S, (Tout*)a.out, a.lse, o_part, lse_part, a.req_status, a.B);
   return cudaGetLastError();
 }
 
@@ -304,8 +331,12 @@ cudaError_t launch_typed(const va_attn_args& a, int S, float* o_part, float* lse
 cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float* lse_part,
                              cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
-  if (a.dtype == VA_F32) return launch_typed<float, float>(a, S, o_part, lse_part, st);
-  return launch_typed<__nv_bfloat16, __nv_bfloat16>(a, S, o_part, lse_part, st);
+  const bool fp8 = (a.flags & VA_FLAG_KV_FP8_E4M3) != 0;
+  if (a.dtype == VA_F32)
+    return fp8 ? launch_typed<float, uint8_t, float>(a, S, o_part, lse_part, st)
+               : launch_typed<float, float, float>(a, S, o_part, lse_part, st);
+  return fp8 ? launch_typed<__nv_bfloat16, uint8_t, __nv_bfloat16>(a, S, o_part, lse_part, st)
+             : launch_typed<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(a, S, o_part, lse_part, st);
 }
 
 }  // namespace va

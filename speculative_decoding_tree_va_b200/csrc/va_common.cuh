@@ -40,6 +40,12 @@ __host__ __device__ __forceinline__ void split_range(int kv_len, int S, int s, i
   *hi = (int)(b < kv_len ? b : kv_len);
 }
 
+// The kernel a va_verify_attn call runs on: bf16 goes to the tensor cores
+// unless the caller asks for CUDA cores or keeps the cache in FP8.
+inline bool uses_tensor_cores(const va_attn_args& a) {
+  return a.dtype == VA_BF16 && !(a.flags & (VA_FLAG_BF16_CUDA_CORES | VA_FLAG_KV_FP8_E4M3));
+}
+
 // Launchers implemented in the .cu files (internal C++ linkage).
 cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
                               int budget, int32_t* parents, int32_t* tokens, int32_t* depth,

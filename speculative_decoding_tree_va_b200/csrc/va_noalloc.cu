@@ -64,7 +64,7 @@ extern "C" int va_verify_attn_noalloc(const va_attn_args* args, va_stream_t stre
   if (S > 1 && need > kScratchBytes) return VA_ERR_UNSUPPORTED;  // larger than the fixed array
 
   cudaStream_t st = (cudaStream_t)stream;
-  const bool tc = args->dtype == VA_BF16 && !(args->flags & VA_FLAG_BF16_CUDA_CORES);
+  const bool tc = va::uses_tensor_cores(*args);
   float* o_part = nullptr;
   float* lse_part = nullptr;
   if (S > 1) {

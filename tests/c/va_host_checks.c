@@ -39,6 +39,18 @@ int main(void) {
   CHECK(va_build_tree_mask(0, 1, VA_MAX_QLEN + 1, 0, 0, 0) == VA_ERR_INVALID_ARG);
   CHECK(va_tree_accept(0, 0, 0, 1, 0, 0, 0, 0, 0) == VA_ERR_INVALID_ARG);
   CHECK(va_merge(0, 0, 0, 1, 1, 1, VA_F32, 0, 0, 0) == VA_ERR_INVALID_ARG);
+
+  /* FP8 cache: a finite, positive scale is required */
+  a.flags = VA_FLAG_KV_FP8_E4M3;
+  a.kv_scale = 0.0f;
+  CHECK(va_num_splits(&a) == -VA_ERR_INVALID_ARG);
+  a.kv_scale = -1.0f;
+  CHECK(va_verify_attn(&a, 0) == VA_ERR_INVALID_ARG);
+  a.kv_scale = 0.4375f;
+  CHECK(va_num_splits(&a) == 1);
+  a.flags |= VA_FLAG_TEST_STALL_MMA;
+  CHECK(va_num_splits(&a) == -VA_ERR_INVALID_ARG);
+  a.flags = 0;
   printf("host checks ok\n");
   return 0;
 }

@@ -66,6 +66,13 @@ def args(**kw):
     # the bounded-wait test hook exists only on the tensor-core path
     (dict(flags=va.VA_FLAG_TEST_STALL_MMA, dtype=va.VA_F32), va.VA_ERR_INVALID_ARG),
     (dict(flags=va.VA_FLAG_TEST_STALL_MMA | va.VA_FLAG_BF16_CUDA_CORES), va.VA_ERR_INVALID_ARG),
+    # FP8 cache: the scale must be finite and positive; no tensor-core test hook
+    (dict(flags=va.VA_FLAG_KV_FP8_E4M3), va.VA_ERR_INVALID_ARG),  # kv_scale left at 0
+    (dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=-0.5), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=float("nan")), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=float("inf")), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_KV_FP8_E4M3 | va.VA_FLAG_TEST_STALL_MMA, kv_scale=0.5),
+     va.VA_ERR_INVALID_ARG),
 ])
 def test_verify_attn_host_checks(lib, bad, status):
     a = args(**bad)
@@ -104,6 +111,21 @@ def test_split_planning_and_workspace(lib):
     s = lib.va_num_splits(ctypes.byref(args(B=4, T=65, max_pages=2050)))
     assert s > 1 and (4 * 33 * s) % 74 >= 0
     assert lib.va_num_splits(ctypes.byref(args(T=66))) == -va.VA_ERR_INVALID_ARG
+
+
+def test_fp8_cache_plans_like_the_cuda_core_path(lib):
+    """An FP8 cache runs on the CUDA-core kernel for both query types, so the
+    auto split count is the CUDA-core planner's (32-row CTAs, 148 slots)."""
+    for dt in (va.VA_BF16, va.VA_F32):
+        for B, T, mp in ((1, 33, 33), (4, 65, 2050), (16, 65, 66), (64, 33, 129)):
+            fp8 = args(dtype=dt, B=B, T=T, max_pages=mp, flags=va.VA_FLAG_KV_FP8_E4M3,
+                       kv_scale=0.4375)
+            cc = args(dtype=va.VA_F32, B=B, T=T, max_pages=mp)
+            assert lib.va_num_splits(ctypes.byref(fp8)) == lib.va_num_splits(ctypes.byref(cc))
+    # the bf16 tensor-core planner differs on a case where the two disagree
+    tc = args(B=4, T=65, max_pages=2050)
+    cc = args(B=4, T=65, max_pages=2050, flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=1.0)
+    assert lib.va_num_splits(ctypes.byref(tc)) != lib.va_num_splits(ctypes.byref(cc))
 
 
 def test_c99_program_uses_the_host_api(tmp_path):

@@ -36,7 +36,7 @@ def run_gpu(va, inp, parents, path, num_splits=1, rows=None):
     req_status = torch.zeros(inp.wl.B, dtype=torch.int32, device="cuda")
     out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
                               d["kv_len"], mask, scale=synth.SCALE, num_splits=num_splits,
-                              flags=flags, req_status=req_status)
+                              flags=flags, req_status=req_status, kv_scale=inp.wl.kv_scale)
     torch.cuda.synchronize()
     assert (req_status.cpu().numpy() == 0).all()
     out = out.float().reshape(-1, synth.D_LATENT)
