@@ -201,7 +201,10 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     bf16 = wl.dtype == "bf16"
     fp8 = wl.kv == "fp8_e4m3"
-    tc = bf16 and not fp8        # the tensor-core kernel; everything else runs on CUDA cores
+    # bf16 queries run on the tensor cores (an FP8 cache is widened first)
+    # unless --cuda-cores asks for the CUDA-core kernel
+    tc = bf16 and not args.cuda_cores
+    vflags = va.VA_FLAG_BF16_CUDA_CORES if (bf16 and args.cuda_cores) else 0
     tdt = torch.bfloat16 if bf16 else torch.float32
 
     def to_dev(a):
@@ -229,7 +232,8 @@ def run_gpu(args):
     tstat = torch.empty(B, device=dev, dtype=torch.int32)
     splits = args.splits if args.splits is not None else wl.splits
     vargs = va.make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, out, lse,
-                         scale=synth.SCALE, num_splits=splits, kv_scale=wl.kv_scale)
+                         scale=synth.SCALE, num_splits=splits, kv_scale=wl.kv_scale,
+                         flags=vflags)
     S = va.num_splits(vargs)
     wbytes = va.workspace_bytes(vargs)
     ws = torch.empty(max(wbytes, 256), device=dev, dtype=torch.uint8) if wbytes else None
@@ -306,7 +310,7 @@ def run_gpu(args):
         st_["args"] = va.make_args(st_["q_nope"], st_["q_pe"], c_kv, k_pe, st_["page_table"],
                                    st_["kv_len"], st_["mask"], st_["out"], st_["lse"],
                                    scale=synth.SCALE, num_splits=splits, workspace=st_["ws"],
-                                   kv_scale=wl.kv_scale)
+                                   kv_scale=wl.kv_scale, flags=vflags)
         sets.append(st_)
     s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "run", "out")}
@@ -390,7 +394,7 @@ def run_gpu(args):
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "pipelining": "2 buffer sets, copy-in / compute / copy-out on 3 streams"},
-        "gpu_launches": args.steps * (2 + (1 if S > 1 else 0)),
+        "gpu_launches": args.steps * (2 + (1 if S > 1 else 0) + (1 if tc and fp8 else 0)),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
@@ -500,6 +504,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cuda-cores", action="store_true",
+                    help="run bf16 queries on the CUDA-core kernel (VA_FLAG_BF16_CUDA_CORES)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

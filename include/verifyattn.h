@@ -187,16 +187,26 @@ typedef struct va_attn_args {
  * subnormal; S.1111.111 is NaN; no infinities; largest magnitude 448).  The
  * cache takes half the bytes of a bf16 one; queries and outputs keep `dtype`
  * (fp32 or bf16).  The pages keep the cache in the model's dtype: this is an
- * addition.  Both query types run on the CUDA-core kernel, which widens every
- * code exactly.  kv_scale must be finite and > 0, else VA_ERR_INVALID_ARG;
- * VA_FLAG_TEST_STALL_MMA is rejected with this flag. */
+ * addition.  bf16 queries run on the tensor-core kernel: a first kernel
+ * widens the pages the batch reads into bf16 scratch pages in the workspace
+ * (every E4M3 value is exactly a bf16 value; slots past kv_len become zeros),
+ * and kv_scale is folded into the score scale and the output normalisation.
+ * fp32 queries (or VA_FLAG_BF16_CUDA_CORES) run on the CUDA-core kernel,
+ * which widens codes to fp32 as it stages them.  kv_scale must be finite and
+ * > 0, else VA_ERR_INVALID_ARG; VA_FLAG_TEST_STALL_MMA is rejected with this
+ * flag. */
 #define VA_FLAG_KV_FP8_E4M3 4
 
 /*
- * Workspace needed by va_verify_attn for these arguments (0 for a single
- * pass).  With S = the split count the call will use, the workspace holds
- * o_part float [S, B, T, H, 512] followed (256-byte aligned) by lse_part
- * float [S, B, T, H]; the layout va_merge reads.  Returns 0 on bad args.
+ * Workspace needed by va_verify_attn for these arguments (0 when none is
+ * needed).  With S = the split count the call will use, the workspace holds,
+ * each part starting on a 256-byte boundary:
+ *   - for S > 1: o_part float [S, B, T, H, 512], then lse_part float
+ *     [S, B, T, H] (the layout va_merge reads);
+ *   - for bf16 queries on the tensor cores with an FP8 cache: the widened
+ *     cache, bf16 [B * max_pages, 64, 512] and [B * max_pages, 64, 64], and
+ *     its page table int32 [B, max_pages].
+ * Returns 0 on bad args.
  */
 size_t va_workspace_bytes(const va_attn_args* args);
 
@@ -255,8 +265,10 @@ int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, in
  * that args->workspace / workspace_bytes are ignored: the split-KV partials
  * live in a fixed array of VA_NOALLOC_SCRATCH_BYTES inside the library.
  *   - Returns VA_ERR_UNSUPPORTED, before launching anything, when the
- *     partials need more than that: S * B * T * H * (512 + 1) floats (each
- *     part rounded up to 256 bytes) must fit.  S = 1 needs no scratch.
+ *     workspace va_verify_attn would need (va_workspace_bytes) exceeds that:
+ *     the partials, S * B * T * H * (512 + 1) floats, and for bf16 queries
+ *     against an FP8 cache the widened pages, B * max_pages * 73,728 bytes
+ *     plus the page table.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any

@@ -12,7 +12,6 @@ constexpr int kSms = 148;  // B200 SM count; the split planner's wave size
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Host-side checks shared by va_verify_attn / va_workspace_bytes.
 int check_args(const va_attn_args* a) {
@@ -23,14 +22,17 @@ int check_args(const va_attn_args* a) {
   if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
   if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA | VA_FLAG_KV_FP8_E4M3))
     return VA_ERR_INVALID_ARG;
-  if ((a->flags & VA_FLAG_TEST_STALL_MMA) && !va::uses_tensor_cores(*a))
-    return VA_ERR_INVALID_ARG;  // only the tensor-core kernel has the hook
+  if ((a->flags & VA_FLAG_TEST_STALL_MMA) &&
+      (!va::uses_tensor_cores(*a) || (a->flags & VA_FLAG_KV_FP8_E4M3)))
+    return VA_ERR_INVALID_ARG;  // only the tensor-core kernel on a bf16 cache has the hook
   if ((a->flags & VA_FLAG_KV_FP8_E4M3) && !(a->kv_scale > 0.f && a->kv_scale <= FLT_MAX))
     return VA_ERR_INVALID_ARG;  // NaN, zero, negative or infinite cache scale
   if (!(a->scale == a->scale)) return VA_ERR_INVALID_ARG;  // NaN scale
   if (a->B == 0) return VA_OK;
   if (a->num_pages < 1 || a->max_pages < 1) return VA_ERR_INVALID_ARG;
   if ((long long)a->num_pages * VA_PAGE_SIZE > 0x7fffffffLL) return VA_ERR_UNSUPPORTED;
+  if (va::widens_fp8_cache(*a) && (long long)a->B * a->max_pages * VA_PAGE_SIZE > 0x7fffffffLL)
+    return VA_ERR_UNSUPPORTED;  // the widened pages are indexed like a pool
   const void* need16[] = {a->q_nope, a->q_pe, a->c_kv, a->k_pe, a->out};
   for (const void* p : need16)
     if (!p || !aligned(p, 16)) return VA_ERR_INVALID_ARG;
@@ -68,14 +70,47 @@ int plan_splits(const va_attn_args* a) {
   return VA_MAX_SPLITS;
 }
 
-size_t part_bytes(const va_attn_args* a, int S, size_t* lse_off) {
-  const size_t rows = (size_t)a->B * a->T * a->H;
-  const size_t o = align_up((size_t)S * rows * VA_D_LATENT * sizeof(float), 256);
-  if (lse_off) *lse_off = o;
-  return o + align_up((size_t)S * rows * sizeof(float), 256);
+}  // namespace
+
+namespace va {
+
+int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(a, S);
+  char* base = static_cast<char*>(ws);
+  float* o_part = S > 1 ? reinterpret_cast<float*>(base + w.o_part) : nullptr;
+  float* lse_part = S > 1 ? reinterpret_cast<float*>(base + w.lse_part) : nullptr;
+  cudaError_t e;
+  if (widens_fp8_cache(a)) {
+    // FP8 cache under bf16 queries: widen the pages the batch reads, then run
+    // the tensor-core kernel on them with the cache scale folded into the
+    // score scale and into the output normalisation.
+    void* wc = base + w.w_ckv;
+    void* wk = base + w.w_kpe;
+    int32_t* wt = reinterpret_cast<int32_t*>(base + w.w_table);
+    e = launch_kv_widen(a, wc, wk, wt, st);
+    if (e != cudaSuccess) return VA_ERR_CUDA;
+    va_attn_args b = a;
+    b.c_kv = wc;
+    b.k_pe = wk;
+    b.page_table = wt;
+    b.num_pages = a.B * a.max_pages;
+    b.scale = a.scale * a.kv_scale;
+    e = launch_attn_tc(b, S, o_part, lse_part, st, a.kv_scale);
+  } else if (uses_tensor_cores(a)) {
+    e = launch_attn_tc(a, S, o_part, lse_part, st, 1.f);
+  } else {
+    e = launch_attn_simt(a, S, o_part, lse_part, st);
+  }
+  if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return VA_ERR_CUDA;
+  if (S > 1) {
+    e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out, a.lse, st);
+    if (e != cudaSuccess) return VA_ERR_CUDA;
+  }
+  return VA_OK;
 }
 
-}  // namespace
+}  // namespace va
 
 extern "C" {
 
@@ -134,38 +169,19 @@ int va_num_splits(const va_attn_args* args) {
 }
 
 size_t va_workspace_bytes(const va_attn_args* args) {
-  if (check_args(args) != VA_OK) return 0;
-  const int S = plan_splits(args);
-  if (S <= 1 || args->B == 0) return 0;
-  return part_bytes(args, S, nullptr);
+  if (check_args(args) != VA_OK || args->B == 0) return 0;
+  return va::workspace_layout(*args, plan_splits(args)).total;
 }
 
 int va_verify_attn(const va_attn_args* args, va_stream_t stream) {
-  int st = check_args(args);
+  const int st = check_args(args);
   if (st != VA_OK) return st;
   if (args->B == 0) return VA_OK;
   const int S = plan_splits(args);
-  float* o_part = nullptr;
-  float* lse_part = nullptr;
-  if (S > 1) {
-    size_t lse_off = 0;
-    const size_t need = part_bytes(args, S, &lse_off);
-    if (!args->workspace || !aligned(args->workspace, 256) || args->workspace_bytes < need)
-      return VA_ERR_INVALID_ARG;
-    o_part = (float*)args->workspace;
-    lse_part = (float*)((char*)args->workspace + lse_off);
-  }
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = va::uses_tensor_cores(*args) ? va::launch_attn_tc(*args, S, o_part, lse_part, s)
-                                         : va::launch_attn_simt(*args, S, o_part, lse_part, s);
-  if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return VA_ERR_CUDA;
-  if (S > 1) {
-    e = va::launch_merge(o_part, lse_part, S, (long long)args->B * args->T * args->H,
-                         args->dtype, args->out, args->lse, s);
-    if (e != cudaSuccess) return VA_ERR_CUDA;
-  }
-  return VA_OK;
+  const size_t need = va::workspace_layout(*args, S).total;
+  if (need && (!args->workspace || !aligned(args->workspace, 256) || args->workspace_bytes < need))
+    return VA_ERR_INVALID_ARG;
+  return va::run_verify(*args, S, args->workspace, (cudaStream_t)stream);
 }
 
 int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,

@@ -68,6 +68,7 @@ struct TcParams {
   int B, H, T, R, max_pages, num_pages, S;
   int stall_mma;  // test hook: issue no tensor-core work (the waits expire)
   float scale_log2;
+  float out_scale;  // multiplies the normalised output (an FP8 cache's scale; else 1)
 };
 
 struct __align__(16) Ctl {
@@ -631,7 +632,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     const float lsumr = lr + c.xsumr[h ^ 1][m];
     const bool bad = !req_ok || c.bad_page || *abort;
     const bool empty = bad || !(lsum > 0.f) || !(lsumr > 0.f) || ntiles == 0;
-    const float inv = empty ? 0.f : 1.f / lsumr;
+    const float inv = empty ? 0.f : p.out_scale / lsumr;
     const float lse = empty ? -INFINITY : (m_used + log2f(lsum)) * kLn2;
     __syncwarp();
     {
@@ -741,7 +742,7 @@ bool encode_2d(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) 
 }  // namespace
 
 cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                           cudaStream_t st) {
+                           cudaStream_t st, float out_scale) {
   if (a.B == 0) return cudaSuccess;
   const long long R = (long long)a.T * a.H;
   const long long rows_total = (long long)a.B * R;
@@ -775,6 +776,7 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   p.S = S;
   p.stall_mma = (a.flags & VA_FLAG_TEST_STALL_MMA) ? 1 : 0;
   p.scale_log2 = a.scale * kLog2e;
+  p.out_scale = out_scale;
   dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)S);
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, tckv3, p);
   return cudaGetLastError();

@@ -40,10 +40,50 @@ __host__ __device__ __forceinline__ void split_range(int kv_len, int S, int s, i
   *hi = (int)(b < kv_len ? b : kv_len);
 }
 
-// The kernel a va_verify_attn call runs on: bf16 goes to the tensor cores
-// unless the caller asks for CUDA cores or keeps the cache in FP8.
+// The kernel a va_verify_attn call runs on: bf16 queries go to the tensor
+// cores unless the caller asks for CUDA cores; fp32 queries to CUDA cores.
 inline bool uses_tensor_cores(const va_attn_args& a) {
-  return a.dtype == VA_BF16 && !(a.flags & (VA_FLAG_BF16_CUDA_CORES | VA_FLAG_KV_FP8_E4M3));
+  return a.dtype == VA_BF16 && !(a.flags & VA_FLAG_BF16_CUDA_CORES);
+}
+
+// A tensor-core call with an FP8 cache first widens the pages it reads into
+// bf16 scratch pages (part of the workspace).
+inline bool widens_fp8_cache(const va_attn_args& a) {
+  return uses_tensor_cores(a) && (a.flags & VA_FLAG_KV_FP8_E4M3);
+}
+
+// Workspace layout of one call: split-KV partials (S > 1), then the widened
+// cache (widens_fp8_cache): bf16 [B * max_pages, 64, 512], bf16
+// [B * max_pages, 64, 64] and an int32 [B, max_pages] page table; every part
+// starts on a 256-byte boundary.  Offsets are in bytes; `total` is 0 when
+// nothing is needed.
+struct WorkspaceLayout {
+  size_t o_part, lse_part, w_ckv, w_kpe, w_table, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S) {
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0};
+  const size_t rows = (size_t)a.B * a.T * a.H;
+  size_t off = 0;
+  if (S > 1) {
+    w.o_part = off;
+    off += align256((size_t)S * rows * kDc * sizeof(float));
+    w.lse_part = off;
+    off += align256((size_t)S * rows * sizeof(float));
+  }
+  if (widens_fp8_cache(a)) {
+    const size_t pages = (size_t)a.B * a.max_pages;
+    w.w_ckv = off;
+    off += align256(pages * kPage * kDc * 2);
+    w.w_kpe = off;
+    off += align256(pages * kPage * kDr * 2);
+    w.w_table = off;
+    off += align256(pages * sizeof(int32_t));
+  }
+  w.total = off;
+  return w;
 }
 
 // Launchers implemented in the .cu files (internal C++ linkage).
@@ -60,6 +100,12 @@ cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float*
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
                          int out_dtype, void* out, float* lse, cudaStream_t st);
 cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                           cudaStream_t st);
+                           cudaStream_t st, float out_scale);
+cudaError_t launch_kv_widen(const va_attn_args& a, void* w_ckv, void* w_kpe, int32_t* w_table,
+                            cudaStream_t st);
+
+// Everything va_verify_attn launches once its arguments are checked and its
+// split count S is known, with the workspace at `ws` laid out as above.
+int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st);
 
 }  // namespace va

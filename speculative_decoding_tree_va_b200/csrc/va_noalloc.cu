@@ -5,9 +5,10 @@
 // verify step: a serving loop whose device memory is planned once at start-up
 // and may not grow, or a latency-critical path where an allocation (which can
 // synchronise the device) is not acceptable.  va_verify_attn needs such a
-// caller to hand over a workspace for the split-KV partials; this entry point
-// instead keeps the partials in a fixed array of this library, so the caller
-// passes only inputs and outputs.
+// caller to hand over a workspace for the split-KV partials (and, for bf16
+// queries against an FP8 cache, the widened cache pages); this entry point
+// instead keeps them in a fixed array of this library, so the caller passes
+// only inputs and outputs.
 //
 // The array has kScratchBytes (VA_NOALLOC_SCRATCH_BYTES) on every device that
 // loads the library, for as long as the process lives.  Every call shares it
@@ -33,8 +34,6 @@ void* g_scratch_addr[kMaxDevices];
 cudaError_t g_scratch_err[kMaxDevices];
 std::once_flag g_scratch_once[kMaxDevices];
 
-size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
 // Device address of the scratch array on the current device, looked up once
 // per device (with that device current) and cached.
 cudaError_t scratch_address(void** addr) {
@@ -53,34 +52,14 @@ cudaError_t scratch_address(void** addr) {
 }  // namespace
 
 extern "C" int va_verify_attn_noalloc(const va_attn_args* args, va_stream_t stream) {
-  // Argument checks and the split count are exactly those of va_verify_attn;
-  // the workspace fields of args are ignored.
+  // Argument checks, the split count and the workspace layout are exactly
+  // those of va_verify_attn; the workspace fields of args are ignored.
   const int S = va_num_splits(args);
   if (S < 0) return -S;
   if (args->B == 0) return VA_OK;
-  const size_t rows = (size_t)args->B * args->T * args->H;
-  const size_t lse_off = align256((size_t)S * rows * VA_D_LATENT * sizeof(float));
-  const size_t need = lse_off + align256((size_t)S * rows * sizeof(float));
-  if (S > 1 && need > kScratchBytes) return VA_ERR_UNSUPPORTED;  // larger than the fixed array
-
-  cudaStream_t st = (cudaStream_t)stream;
-  const bool tc = va::uses_tensor_cores(*args);
-  float* o_part = nullptr;
-  float* lse_part = nullptr;
-  if (S > 1) {
-    void* base = nullptr;
-    if (scratch_address(&base) != cudaSuccess) return VA_ERR_CUDA;
-    o_part = (float*)base;
-    lse_part = (float*)((char*)base + lse_off);
-  }
-  cudaError_t e = tc ? va::launch_attn_tc(*args, S, o_part, lse_part, st)
-                     : va::launch_attn_simt(*args, S, o_part, lse_part, st);
-  if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return VA_ERR_CUDA;
-  if (S > 1) {
-    e = va::launch_merge(o_part, lse_part, S, (long long)rows, args->dtype, args->out, args->lse,
-                         st);
-    if (e != cudaSuccess) return VA_ERR_CUDA;
-  }
-  return VA_OK;
+  const size_t need = va::workspace_layout(*args, S).total;
+  if (need > kScratchBytes) return VA_ERR_UNSUPPORTED;  // larger than the fixed array
+  void* base = nullptr;
+  if (need && scratch_address(&base) != cudaSuccess) return VA_ERR_CUDA;
+  return va::run_verify(*args, S, base, (cudaStream_t)stream);
 }

@@ -47,7 +47,12 @@ int main(void) {
   a.kv_scale = -1.0f;
   CHECK(va_verify_attn(&a, 0) == VA_ERR_INVALID_ARG);
   a.kv_scale = 0.4375f;
+  a.num_splits = 1;
   CHECK(va_num_splits(&a) == 1);
+  CHECK(va_workspace_bytes(&a) > 0);   /* bf16 on tensor cores: the widened pages */
+  a.dtype = VA_F32;
+  CHECK(va_workspace_bytes(&a) == 0);  /* fp32 on CUDA cores widens while staging */
+  a.dtype = VA_BF16;
   a.flags |= VA_FLAG_TEST_STALL_MMA;
   CHECK(va_num_splits(&a) == -VA_ERR_INVALID_ARG);
   a.flags = 0;

@@ -113,19 +113,36 @@ def test_split_planning_and_workspace(lib):
     assert lib.va_num_splits(ctypes.byref(args(T=66))) == -va.VA_ERR_INVALID_ARG
 
 
-def test_fp8_cache_plans_like_the_cuda_core_path(lib):
-    """An FP8 cache runs on the CUDA-core kernel for both query types, so the
-    auto split count is the CUDA-core planner's (32-row CTAs, 148 slots)."""
+def test_fp8_cache_split_planning_and_workspace(lib):
+    """An FP8 cache keeps the query type's kernel (bf16: tensor cores, fp32: CUDA
+    cores), so the auto split count is that kernel's; bf16 on the tensor cores
+    adds the widened pages to the workspace."""
+    fp8 = dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=0.4375)
     for dt in (va.VA_BF16, va.VA_F32):
         for B, T, mp in ((1, 33, 33), (4, 65, 2050), (16, 65, 66), (64, 33, 129)):
-            fp8 = args(dtype=dt, B=B, T=T, max_pages=mp, flags=va.VA_FLAG_KV_FP8_E4M3,
-                       kv_scale=0.4375)
-            cc = args(dtype=va.VA_F32, B=B, T=T, max_pages=mp)
-            assert lib.va_num_splits(ctypes.byref(fp8)) == lib.va_num_splits(ctypes.byref(cc))
-    # the bf16 tensor-core planner differs on a case where the two disagree
-    tc = args(B=4, T=65, max_pages=2050)
-    cc = args(B=4, T=65, max_pages=2050, flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=1.0)
+            a = args(dtype=dt, B=B, T=T, max_pages=mp, **fp8)
+            plain = args(dtype=dt, B=B, T=T, max_pages=mp)
+            assert lib.va_num_splits(ctypes.byref(a)) == lib.va_num_splits(ctypes.byref(plain))
+    # the two planners differ here, so the routing is visible
+    tc = args(B=4, T=65, max_pages=2050, **fp8)
+    cc = args(B=4, T=65, max_pages=2050, flags=fp8["flags"] | va.VA_FLAG_BF16_CUDA_CORES,
+              kv_scale=0.4375)
     assert lib.va_num_splits(ctypes.byref(tc)) != lib.va_num_splits(ctypes.byref(cc))
+    # single pass: only the widened cache (B * max_pages pages) and its page table
+    a = args(num_splits=1, **fp8)                     # B = 2, max_pages = 50
+    pages = 2 * 50
+    up = lambda x: (x + 255) // 256 * 256
+    want = up(pages * 64 * 512 * 2) + up(pages * 64 * 64 * 2) + up(pages * 4)
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == want
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, dtype=va.VA_F32, **fp8))) == 0
+    # with splits the partials come first
+    a = args(num_splits=4, **fp8)
+    rows = 2 * 33 * 64
+    parts = up(4 * rows * 512 * 4) + up(4 * rows * 4)
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == parts + want
+    # the no-allocation entry point refuses, before any launch, what its fixed array cannot hold
+    big = args(B=64, max_pages=129, num_splits=1, **fp8)
+    assert lib.va_verify_attn_noalloc(ctypes.byref(big), None) == va.VA_ERR_UNSUPPORTED
 
 
 def test_c99_program_uses_the_host_api(tmp_path):

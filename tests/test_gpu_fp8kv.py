@@ -1,11 +1,12 @@
 """GPU parity of va_verify_attn with an FP8 E4M3 latent cache
 (VA_FLAG_KV_FP8_E4M3) against the fp64 oracle, which decodes the codes itself.
 
-Both query types run on the CUDA-core kernel.  Decoding is exact on both sides,
-so only the kernel's fp32 arithmetic differs from the oracle and the bars are
-those of the query dtype: fp32 max_abs <= 1e-5; bf16 out <= 1e-2, lse <= 1e-3.
-Paths "tc" and "cc" differ only in VA_FLAG_BF16_CUDA_CORES, which an FP8 cache
-makes moot; both are run to check the routing.
+Paths: "f32" (fp32 queries, CUDA-core kernel widening codes as it stages
+them), "tc" (bf16 queries: the pages are widened into bf16 scratch pages, then
+the tensor-core kernel runs with the cache scale folded in) and "cc" (bf16
+queries on the CUDA-core kernel, VA_FLAG_BF16_CUDA_CORES).  Widening is exact
+on every path and the oracle decodes the codes itself, so the bars are those
+of the query dtype: fp32 max_abs <= 1e-5; bf16 out <= 1e-2, lse <= 1e-3.
 """
 import dataclasses
 
@@ -119,8 +120,8 @@ def test_fp8kv_bad_page_is_flagged(va, dtype, path):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_uint8_cache_noalloc_and_flag_agree(va, dtype):
-    """A uint8 cache, a float8_e4m3fn cache and va_verify_attn_noalloc give the
-    same bits (one kernel, one split plan)."""
+    """A uint8 cache, a float8_e4m3fn cache and va_verify_attn_noalloc (whose
+    fixed array then also holds the widened pages for bf16) give the same bits."""
     import torch
     inp = fp8_inputs(dtype, B=2, H=8, P=900, budget=12)
     parents = trees_for(inp)["parent"]
