@@ -61,6 +61,7 @@ enum va_dtype { VA_F32 = 0, VA_BF16 = 1 };
 #define VA_MAX_TOPK 16    /* widest drafter top-k the builder accepts     */
 #define VA_SPLIT_ALIGN 256/* split-KV chunk granularity, in keys          */
 #define VA_MAX_SPLITS 64
+#define VA_MAX_BATCH 65535 /* requests per va_verify_attn call              */
 
 /* Largest tree-verify query length T (root included): 65.  The pages'
  * library reports the same limit when it loads ("Verified lib loads
@@ -231,9 +232,12 @@ int va_num_splits(const va_attn_args* args);
  * and va_merge combines them on the same stream.
  * bf16 runs on tensor cores with fp32 accumulation; fp32, and any call with
  * an FP8 cache (VA_FLAG_KV_FP8_E4M3), on CUDA cores.
- * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, B >= 0.  Slots past
+ * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, 0 <= B <= VA_MAX_BATCH
+ * (larger batches: VA_ERR_UNSUPPORTED; split them across calls).  Slots past
  * kv_len in a request's last page may hold any finite values (they are
- * multiplied by exact zeros; NaN or Inf there would propagate).
+ * multiplied by exact zeros; NaN or Inf there would propagate); with an FP8
+ * cache they may hold any codes, NaN included (both FP8 routes replace them
+ * by zeros before any product).
  */
 int va_verify_attn(const va_attn_args* args, va_stream_t stream);
 

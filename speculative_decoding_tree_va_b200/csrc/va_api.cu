@@ -19,6 +19,7 @@ int check_args(const va_attn_args* a) {
   if (a->dtype != VA_F32 && a->dtype != VA_BF16) return VA_ERR_INVALID_ARG;
   if (a->B < 0 || a->H < 1 || a->T < 1 || a->T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
   if (a->page_size != VA_PAGE_SIZE) return VA_ERR_UNSUPPORTED;
+  if (a->B > VA_MAX_BATCH) return VA_ERR_UNSUPPORTED;  // the launches' request axis (grid y)
   if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
   if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA | VA_FLAG_KV_FP8_E4M3))
     return VA_ERR_INVALID_ARG;

@@ -63,6 +63,7 @@ def args(**kw):
     (dict(flags=8), va.VA_ERR_INVALID_ARG), (dict(num_pages=0), va.VA_ERR_INVALID_ARG),
     (dict(num_splits=4), va.VA_ERR_INVALID_ARG),  # split without a workspace
     (dict(scale=float("nan")), va.VA_ERR_INVALID_ARG),
+    (dict(B=65536), va.VA_ERR_UNSUPPORTED),     # beyond the launches' request axis
     # the bounded-wait test hook exists only on the tensor-core path
     (dict(flags=va.VA_FLAG_TEST_STALL_MMA, dtype=va.VA_F32), va.VA_ERR_INVALID_ARG),
     (dict(flags=va.VA_FLAG_TEST_STALL_MMA | va.VA_FLAG_BF16_CUDA_CORES), va.VA_ERR_INVALID_ARG),
