@@ -388,7 +388,8 @@ def run_gpu(args):
                      "traffic": traffic,
                      "peak_source": (f"{peak_src} bf16 dense (burst); sustained {tc_sust}" if tc else
                                      "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz"),
-                     "kernel": "attn_tc_kernel" if tc else "attn_simt_kernel",
+                     "kernel": (("kv_widen_kernel + attn_tc_kernel" if fp8 else "attn_tc_kernel")
+                                if tc else "attn_simt_kernel"),
                      "kernel_us": round(attn_ms * 1e3, 1), "roofline_us": round(roof_us, 1),
                      "frac_of_step_roofline": round(roof_us / (ms_step * 1e3), 4)},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
