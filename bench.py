@@ -244,7 +244,9 @@ def run_gpu(args):
     sptr = va._stream(stream)
     import ctypes
 
-    def step(ev_a=None, ev_b=None):
+    def step(ev_a=None, ev_b=None, ev_s=None):
+        if ev_s is not None:
+            ev_s.record(stream)
         r = lib.va_build_tree_mask(ctypes.c_void_p(parents.data_ptr()), B, T,
                                    ctypes.c_void_p(mask.data_ptr()),
                                    ctypes.c_void_p(tstat.data_ptr()), sptr)
@@ -261,23 +263,27 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     # timed region: K back-to-back steps, inputs (> 126 MB L2) resident in HBM
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with Clocks(local) as clk:
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
         t0.record(stream)
-        for a, b in evs:
-            step(a, b)
+        for a, b, c in evs:
+            step(a, b, c)
         t1.record(stream)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
     ms_total = t0.elapsed_time(t1)
     ms_total = max_over_ranks(ms_total, dist)
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in evs]))
+    # per-step spread: step i runs from its first event to the next step's
+    # first event (the last one to the end of the region)
+    starts = [c for _, _, c in evs] + [t1]
+    step_ms = [starts[i].elapsed_time(starts[i + 1]) for i in range(args.steps)]
     ms_step = ms_total / args.steps
     world = args.gpus
     value = flops * world / (ms_step * 1e-3) / 1e12
@@ -366,6 +372,15 @@ def run_gpu(args):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     roof_us = max(flops / ((tc_peak if tc else FP32_FFMA_PEAK) * 1e12), alg_bytes / (hbm * 1e9)) * 1e6
     clocks = clk.summary()
+    # the split-KV long prefix and the deep-tree batch, timed in the same
+    # process beside the headline (one GPU only; replicas skip them)
+    others = None
+    if world == 1 and not args.no_other_workloads and not args.cuda_cores:
+        others = {}
+        for name, sp in OTHER_WORKLOADS:
+            if name == wl.name and sp == S:
+                continue
+            others[f"{name} S={sp}"] = time_workload(va, name, sp, dev, steps=10, warmup=3)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
@@ -379,6 +394,9 @@ def run_gpu(args):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "us_per_step": round(ms_step * 1e3, 1),
+        "us_per_step_spread": {"min": round(min(step_ms) * 1e3, 1),
+                               "median": round(float(np.median(step_ms)) * 1e3, 1),
+                               "max": round(max(step_ms) * 1e3, 1)},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if tc else "f32", "data": "synthetic (seeded; no dataset or weights)",
         "config": config_of(wl, S, world, flops, alg_bytes),
@@ -395,11 +413,207 @@ def run_gpu(args):
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "pipelining": "2 buffer sets, copy-in / compute / copy-out on 3 streams"},
-        "gpu_launches": args.steps * (2 + (1 if S > 1 else 0) + (1 if tc and fp8 else 0)),
+        "gpu_launches": args.steps * launches_per_step(tc, fp8, S),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
+    if others:
+        line["other_workloads"] = others
     print(json.dumps(line), flush=True)
+
+
+OTHER_WORKLOADS = [("bf16-long-prefix", 16), ("bf16-long-prefix", 64), ("bf16-deep", 1)]
+
+
+def run_sharded(args):
+    """One batch for the whole job, its split-KV partition shared out across the GPUs.
+
+    Every rank holds the same batch; rank r computes its block of the S splits
+    (va_verify_attn_partials), merges them locally, the ranks' partials are
+    all-gathered (NCCL), and rank 0 merges them into out / lse.  Strong
+    scaling: the work per step is fixed, `value` = its flops / the slowest
+    rank's step time.  With one GPU the gather is skipped."""
+    import ctypes
+
+    import torch
+    import speculative_decoding_tree_va_b200 as va
+    from speculative_decoding_tree_va_b200.shard import ShardedStep
+
+    rank, local, dist = dist_setup(args.gpus)
+    world = args.gpus
+    wl = synth.WORKLOADS[args.workload]
+    S = args.splits if args.splits is not None else wl.splits
+    if S < 1:
+        raise SystemExit("--shard-prefix needs an explicit split count (--splits)")
+    inp = synth.make_inputs(wl)                      # the same batch on every rank
+    dev = torch.device("cuda", local)
+    bf16 = wl.dtype == "bf16"
+    tdt = torch.bfloat16 if bf16 else torch.float32
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.int16).view(torch.bfloat16) if bf16 else t).to(dev)
+
+    parents, _, depth, _ = va.build_tree(torch.from_numpy(inp.lp).to(dev),
+                                         torch.from_numpy(inp.tok).to(dev), wl.budget)
+    flops, alg_bytes = work(inp, depth.cpu().numpy())
+    B, T, H = wl.B, wl.T, wl.H
+    q_nope, q_pe, c_kv, k_pe = (to_dev(a) for a in (inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe))
+    page_table = torch.from_numpy(inp.page_table).to(dev)
+    kv_len = torch.from_numpy(inp.kv_len).to(dev)
+    mask = torch.empty(B, T, (T + 63) // 64, device=dev, dtype=torch.int64)
+    tstat = torch.empty(B, device=dev, dtype=torch.int32)
+    out = torch.empty(B, T, H, synth.D_LATENT, device=dev, dtype=tdt)
+    lse = torch.empty(B, T, H, device=dev, dtype=torch.float32)
+    vargs = va.make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, out, lse,
+                         scale=synth.SCALE, num_splits=S)
+    lib = va.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sptr = va._stream(stream)
+
+    class _One:  # one rank: the gather is the identity
+        @staticmethod
+        def all_gather_into_tensor(o_all, o, group=None):
+            o_all.copy_(o.reshape(o_all.shape))
+
+    sharded = ShardedStep(va, vargs, rank, world, dist if dist is not None else _One(), dev)
+
+    def step():
+        if lib.va_build_tree_mask(ctypes.c_void_p(parents.data_ptr()), B, T,
+                                  ctypes.c_void_p(mask.data_ptr()),
+                                  ctypes.c_void_p(tstat.data_ptr()), sptr):
+            raise RuntimeError("va_build_tree_mask failed")
+        sharded()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / args.steps, dist) if dist is not None \
+        else t0.elapsed_time(t1) / args.steps
+    # rank 0 checks the sharded result against the one-GPU call of the same batch
+    check = None
+    if rank == 0:
+        out1, lse1 = va.verify_attn(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask,
+                                    scale=synth.SCALE, num_splits=S)
+        torch.cuda.synchronize()
+        fin = torch.isfinite(lse1)
+        check = {"out_max_abs_vs_one_gpu": float((out.float() - out1.float()).abs().max()),
+                 "lse_max_abs_vs_one_gpu": float((lse[fin] - lse1[fin]).abs().max())}
+    clocks = clk.summary()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    _, tc_peak, tc_sust, peak_src = peaks()
+    value = flops / (ms_step * 1e-3) / 1e12
+    cfg = config_of(wl, S, world, flops, alg_bytes)
+    cfg["parallelism"] = f"split-KV partition of one batch across {world} GPU(s)"
+    rows = B * T * H
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "us_per_step": round(ms_step * 1e3, 1), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16" if bf16 else "f32",
+        "data": "synthetic (seeded; no dataset or weights)", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": round(value / world, 2), "per": "GPU",
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": round(value / world / tc_peak, 4),
+                     "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)"},
+        "exchange_bytes_per_rank": rows * (synth.D_LATENT + 1) * 4,
+        "check": check, "clocks": clocks,
+        "gpu_launches": args.steps * (1 + 1 + 1 + (1 if sharded.count > 1 else 0) + 1),
+        "e2e": {"value": None, "note": "not measured in the sharded mode (device-resident batch)"},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def launches_per_step(tc: bool, fp8: bool, S: int) -> int:
+    """Library kernels one step launches: the tree mask, the request order
+    (tensor cores), the FP8 widening pass (tensor cores with an FP8 cache),
+    the attention kernel, and the merge when split."""
+    return 2 + (1 if tc else 0) + (1 if tc and fp8 else 0) + (1 if S > 1 else 0)
+
+
+def time_workload(va, name: str, splits: int, dev, steps: int = 10, warmup: int = 3) -> dict:
+    """Device time of mask + verify steps of one more workload (CUDA events, per step)."""
+    import ctypes
+
+    import torch
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_inputs(wl)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.int16).view(torch.bfloat16) if wl.dtype == "bf16" else t).to(dev)
+
+    parents, _, depth, _ = va.build_tree(torch.from_numpy(inp.lp).to(dev),
+                                         torch.from_numpy(inp.tok).to(dev), wl.budget)
+    flops, alg_bytes = work(inp, depth.cpu().numpy())
+    B, T, H = wl.B, wl.T, wl.H
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    out = torch.empty(B, T, H, synth.D_LATENT, device=dev, dtype=tdt)
+    lse = torch.empty(B, T, H, device=dev, dtype=torch.float32)
+    mask = torch.empty(B, T, (T + 63) // 64, device=dev, dtype=torch.int64)
+    tstat = torch.empty(B, device=dev, dtype=torch.int32)
+    q_nope, q_pe, c_kv, k_pe = (to_dev(a) for a in (inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe))
+    del inp.c_kv, inp.k_pe
+    page_table = torch.from_numpy(inp.page_table).to(dev)
+    kv_len = torch.from_numpy(inp.kv_len).to(dev)
+    vargs = va.make_args(q_nope, q_pe, c_kv, k_pe, page_table, kv_len, mask, out, lse,
+                         scale=synth.SCALE, num_splits=splits)
+    S = va.num_splits(vargs)
+    wbytes = va.workspace_bytes(vargs)
+    ws = torch.empty(max(wbytes, 256), device=dev, dtype=torch.uint8)
+    vargs.workspace, vargs.workspace_bytes = ws.data_ptr(), wbytes
+    lib = va.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sptr = va._stream(stream)
+
+    def step():
+        r = lib.va_build_tree_mask(ctypes.c_void_p(parents.data_ptr()), B, T,
+                                   ctypes.c_void_p(mask.data_ptr()),
+                                   ctypes.c_void_p(tstat.data_ptr()), sptr)
+        r |= lib.va_verify_attn(ctypes.byref(vargs), sptr)
+        if r:
+            raise RuntimeError("library call failed")
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    _, tc_peak, _, _ = peaks()
+    mean = float(np.mean(ms))
+    res = {"B": B, "H": H, "T": T, "prefix": list(wl.P) if isinstance(wl.P, tuple) else wl.P,
+           "num_splits": S, "steps": steps,
+           "us_per_step": round(mean * 1e3, 1),
+           "us_per_step_spread": {"min": round(min(ms) * 1e3, 1),
+                                  "median": round(float(np.median(ms)) * 1e3, 1),
+                                  "max": round(max(ms) * 1e3, 1)},
+           "tflops": round(flops / (mean * 1e-3) / 1e12, 2),
+           "frac": round(flops / (mean * 1e-3) / 1e12 / tc_peak, 4),
+           "gflop_per_step": round(flops / 1e9, 2), "alg_mb_per_step": round(alg_bytes / 1e6, 1),
+           "l2": "inputs larger than the 126 MB L2, no flush" if alg_bytes > 126e6 else
+                 "inputs fit in L2 (warm)"}
+    del q_nope, q_pe, c_kv, k_pe, ws, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def host_cpu():
@@ -505,12 +719,19 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the long-prefix and deep-tree figures printed beside the headline")
+    ap.add_argument("--shard-prefix", action="store_true",
+                    help="shard the workload's split-KV partition across the GPUs (one batch "
+                         "for the whole job: strong scaling)")
     ap.add_argument("--cuda-cores", action="store_true",
                     help="run bf16 queries on the CUDA-core kernel (VA_FLAG_BF16_CUDA_CORES)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard_prefix:
+        run_sharded(args)
     else:
         run_gpu(args)
 

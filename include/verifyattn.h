@@ -161,7 +161,7 @@ typedef struct va_attn_args {
                          or a page index is out of range (rows written as 0 /
                          -inf)                                                 */
   int num_splits;     /* 0 = auto, 1 = single pass, 2..64 = split-KV + merge    */
-  void* workspace;    /* [device] split-KV partials, >= va_workspace_bytes()    */
+  void* workspace;    /* [device] >= va_workspace_bytes(), 256-byte aligned     */
   size_t workspace_bytes;
   int flags;          /* VA_FLAG_* below                                        */
   float kv_scale;     /* with VA_FLAG_KV_FP8_E4M3: the value of one cache unit
@@ -202,6 +202,9 @@ typedef struct va_attn_args {
  * Workspace needed by va_verify_attn for these arguments (0 when none is
  * needed).  With S = the split count the call will use, the workspace holds,
  * each part starting on a 256-byte boundary:
+ *   - for bf16 queries on the tensor cores: the requests' longest-first
+ *     order, int32 [B] (written by the call itself; the longest requests are
+ *     scheduled first so the launch does not end on one long request);
  *   - for S > 1: o_part float [S, B, T, H, 512], then lse_part float
  *     [S, B, T, H] (the layout va_merge reads);
  *   - for bf16 queries on the tensor cores with an FP8 cache: the widened
@@ -240,6 +243,33 @@ int va_num_splits(const va_attn_args* args);
  * by zeros before any product).
  */
 int va_verify_attn(const va_attn_args* args, va_stream_t stream);
+
+/*
+ * Split-KV partials of some of the splits, without the merge: the per-GPU
+ * step of sharding one long prefix across GPUs (the flash+merge production
+ * note, page "The Milestone Commit...", section "How Decisions Were Made":
+ * each GPU computes some of the flash-decode chunks, their partials are
+ * gathered to one GPU, and va_merge combines them there).
+ *
+ *   args        as for va_verify_attn, with args->num_splits = S, 1 <= S <=
+ *               64, given explicitly (0 is rejected: every participant must
+ *               use the same partition); out and lse are not used (may be
+ *               NULL).  The workspace must hold va_workspace_bytes() of the
+ *               same arguments with num_splits = 1 (the request order, and
+ *               the widened pages for bf16 queries with an FP8 cache).
+ *   split_first, split_count
+ *               the splits [split_first, split_first + split_count) of the
+ *               S-way partition va_verify_attn defines; 0 <= split_first,
+ *               1 <= split_count, split_first + split_count <= S
+ *   o_part      [device] float [split_count, B, T, H, 512]  out: normalised
+ *               partial outputs, 16-byte aligned
+ *   lse_part    [device] float [split_count, B, T, H]  out: partial lse
+ *               (-inf for a split with no visible key)
+ * Partial c holds split split_first + c.  va_merge over all S partials gives
+ * va_verify_attn's result (up to the rounding of a different association).
+ */
+int va_verify_attn_partials(const va_attn_args* args, int split_first, int split_count,
+                            float* o_part, float* lse_part, va_stream_t stream);
 
 /*
  * Merge of split-KV partials (the flash+merge production note, page "The

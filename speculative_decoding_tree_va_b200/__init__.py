@@ -27,7 +27,8 @@ D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 
 EXPORTS = ("va_max_qlen", "va_status_string", "va_build_tree", "va_build_tree_mask",
            "va_workspace_bytes", "va_num_splits", "va_verify_attn", "va_merge",
-           "va_device_timeouts", "va_verify_attn_noalloc", "va_tree_accept")
+           "va_device_timeouts", "va_verify_attn_noalloc", "va_tree_accept",
+           "va_verify_attn_partials")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -84,6 +85,8 @@ def load_library(path: Optional[str] = None):
     lib.va_tree_accept.restype = I
     lib.va_verify_attn_noalloc.argtypes = [ctypes.POINTER(VaAttnArgs), V]
     lib.va_verify_attn_noalloc.restype = I
+    lib.va_verify_attn_partials.argtypes = [ctypes.POINTER(VaAttnArgs), I, I, V, V, V]
+    lib.va_verify_attn_partials.restype = I
     if path is None:
         _lib = lib
     return lib
@@ -234,6 +237,23 @@ def verify_attn_noalloc(args: VaAttnArgs, stream=None):
     array instead of a workspace (for callers that cannot allocate)."""
     _check(load_library().va_verify_attn_noalloc(ctypes.byref(args), _stream(stream)),
            "va_verify_attn_noalloc")
+
+
+def partials_workspace_bytes(args: VaAttnArgs) -> int:
+    """Workspace of va_verify_attn_partials: that of the same call with one split."""
+    one = VaAttnArgs.from_buffer_copy(args)
+    one.num_splits = 1
+    return workspace_bytes(one)
+
+
+def verify_attn_partials(args: VaAttnArgs, split_first: int, split_count: int, o_part, lse_part,
+                         stream=None):
+    """va_verify_attn_partials: splits [split_first, split_first + split_count) of the
+    args.num_splits-way partition into o_part float [count, B, T, H, 512] and
+    lse_part float [count, B, T, H] (cuda tensors), no merge."""
+    _check(load_library().va_verify_attn_partials(ctypes.byref(args), split_first, split_count,
+                                                  _ptr(o_part), _ptr(lse_part), _stream(stream)),
+           "va_verify_attn_partials")
 
 
 def merge(o_part, lse_part, out_dtype, stream=None):

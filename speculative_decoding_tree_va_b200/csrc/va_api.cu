@@ -1,6 +1,7 @@
 // C ABI of libverifyattn: argument checks, split planning, dispatch.
 // Every entry point validates on the host and returns a va_status before
 // launching anything; the caller owns all device memory.
+#include <atomic>
 #include <cfloat>
 #include <cstdio>
 
@@ -8,13 +9,35 @@
 
 namespace {
 
-constexpr int kSms = 148;  // B200 SM count; the split planner's wave size
+constexpr int kDefaultSms = 148;  // B200; used when no device can be queried
+constexpr int kMaxDevices = 128;
+std::atomic<int> g_sm_count[kMaxDevices];  // 0 = not looked up yet
+
+// SM count of the current device (the split planner's wave size), looked up
+// once per device.  Without a usable device (host-only use of the planner)
+// it is the B200's 148; the runtime error that lookup leaves is cleared.
+int sm_count() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return kDefaultSms;
+  }
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2) {
+    (void)cudaGetLastError();
+    return kDefaultSms;
+  }
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 
-// Host-side checks shared by va_verify_attn / va_workspace_bytes.
-int check_args(const va_attn_args* a) {
+// Host-side checks shared by va_verify_attn / va_workspace_bytes.  A
+// partials-only call (va_verify_attn_partials) writes neither out nor lse.
+int check_args(const va_attn_args* a, bool needs_out = true) {
   if (!a) return VA_ERR_INVALID_ARG;
   if (a->dtype != VA_F32 && a->dtype != VA_BF16) return VA_ERR_INVALID_ARG;
   if (a->B < 0 || a->H < 1 || a->T < 1 || a->T > VA_MAX_QLEN) return VA_ERR_INVALID_ARG;
@@ -34,13 +57,14 @@ int check_args(const va_attn_args* a) {
   if ((long long)a->num_pages * VA_PAGE_SIZE > 0x7fffffffLL) return VA_ERR_UNSUPPORTED;
   if (va::widens_fp8_cache(*a) && (long long)a->B * a->max_pages * VA_PAGE_SIZE > 0x7fffffffLL)
     return VA_ERR_UNSUPPORTED;  // the widened pages are indexed like a pool
-  const void* need16[] = {a->q_nope, a->q_pe, a->c_kv, a->k_pe, a->out};
+  const void* need16[] = {a->q_nope, a->q_pe, a->c_kv, a->k_pe};
   for (const void* p : need16)
     if (!p || !aligned(p, 16)) return VA_ERR_INVALID_ARG;
+  if (needs_out && (!a->out || !aligned(a->out, 16))) return VA_ERR_INVALID_ARG;
   if (!a->page_table || !aligned(a->page_table, 4)) return VA_ERR_INVALID_ARG;
   if (!a->kv_len || !aligned(a->kv_len, 4)) return VA_ERR_INVALID_ARG;
   if (!a->tree_mask || !aligned(a->tree_mask, 8)) return VA_ERR_INVALID_ARG;
-  if (!a->lse || !aligned(a->lse, 4)) return VA_ERR_INVALID_ARG;
+  if (needs_out && (!a->lse || !aligned(a->lse, 4))) return VA_ERR_INVALID_ARG;
   if (a->req_status && !aligned(a->req_status, 4)) return VA_ERR_INVALID_ARG;
   return VA_OK;
 }
@@ -54,12 +78,13 @@ int plan_splits(const va_attn_args* a) {
   if (a->B == 0) return 1;
   const long long rows = (long long)a->T * a->H;
   long long units_per_split, slots;
+  const int sms = sm_count();
   if (va::uses_tensor_cores(*a)) {
     units_per_split = (long long)a->B * ((rows + 127) / 128);  // CTA pairs
-    slots = kSms / 2;
+    slots = sms / 2;
   } else {
     units_per_split = (long long)a->B * ((rows + 31) / 32);
-    slots = kSms;
+    slots = sms;
   }
   const long long keys = (long long)a->max_pages * VA_PAGE_SIZE;
   for (int S = 1; S <= VA_MAX_SPLITS; S *= 2) {
@@ -75,12 +100,21 @@ int plan_splits(const va_attn_args* a) {
 
 namespace va {
 
-int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
-  const WorkspaceLayout w = workspace_layout(a, S);
-  char* base = static_cast<char*>(ws);
-  float* o_part = S > 1 ? reinterpret_cast<float*>(base + w.o_part) : nullptr;
-  float* lse_part = S > 1 ? reinterpret_cast<float*>(base + w.lse_part) : nullptr;
+namespace {
+
+// The attention launches of one call (after the FP8 widening pass and the
+// request order, when they apply): splits sp of the partition, partials to
+// o_part / lse_part (nullptr: a single split writing out / lse directly).
+int launch_attention(const va_attn_args& a, SplitRange sp, const WorkspaceLayout& w, char* base,
+                     float* o_part, float* lse_part, cudaStream_t st) {
   cudaError_t e;
+  const int32_t* order = nullptr;
+  if (uses_tensor_cores(a)) {
+    int32_t* ord = reinterpret_cast<int32_t*>(base + w.order);
+    e = launch_request_order(a.kv_len, a.B, ord, st);
+    if (e != cudaSuccess) return VA_ERR_CUDA;
+    order = ord;
+  }
   if (widens_fp8_cache(a)) {
     // FP8 cache under bf16 queries: widen the pages the batch reads, then run
     // the tensor-core kernel on them with the cache scale folded into the
@@ -96,19 +130,38 @@ int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
     b.page_table = wt;
     b.num_pages = a.B * a.max_pages;
     b.scale = a.scale * a.kv_scale;
-    e = launch_attn_tc(b, S, o_part, lse_part, st, a.kv_scale);
+    e = launch_attn_tc(b, sp, order, o_part, lse_part, st, a.kv_scale);
   } else if (uses_tensor_cores(a)) {
-    e = launch_attn_tc(a, S, o_part, lse_part, st, 1.f);
+    e = launch_attn_tc(a, sp, order, o_part, lse_part, st, 1.f);
   } else {
-    e = launch_attn_simt(a, S, o_part, lse_part, st);
+    e = launch_attn_simt(a, sp, o_part, lse_part, st);
   }
   if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return VA_ERR_CUDA;
+  return VA_OK;
+}
+
+}  // namespace
+
+int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(a, S);
+  char* base = static_cast<char*>(ws);
+  float* o_part = S > 1 ? reinterpret_cast<float*>(base + w.o_part) : nullptr;
+  float* lse_part = S > 1 ? reinterpret_cast<float*>(base + w.lse_part) : nullptr;
+  const int r = launch_attention(a, SplitRange{S, 0, S}, w, base, o_part, lse_part, st);
+  if (r != VA_OK) return r;
   if (S > 1) {
-    e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out, a.lse, st);
+    cudaError_t e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out,
+                                 a.lse, st);
     if (e != cudaSuccess) return VA_ERR_CUDA;
   }
   return VA_OK;
+}
+
+int run_partials(const va_attn_args& a, SplitRange sp, void* ws, float* o_part, float* lse_part,
+                 cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(a, sp.S, false);
+  return launch_attention(a, sp, w, static_cast<char*>(ws), o_part, lse_part, st);
 }
 
 }  // namespace va
@@ -183,6 +236,24 @@ int va_verify_attn(const va_attn_args* args, va_stream_t stream) {
   if (need && (!args->workspace || !aligned(args->workspace, 256) || args->workspace_bytes < need))
     return VA_ERR_INVALID_ARG;
   return va::run_verify(*args, S, args->workspace, (cudaStream_t)stream);
+}
+
+int va_verify_attn_partials(const va_attn_args* args, int split_first, int split_count,
+                            float* o_part, float* lse_part, va_stream_t stream) {
+  const int st = check_args(args, false);
+  if (st != VA_OK) return st;
+  const int S = args->num_splits;
+  if (S < 1) return VA_ERR_INVALID_ARG;  // the partition must be explicit
+  if (split_first < 0 || split_count < 1 || split_first > S - split_count)
+    return VA_ERR_INVALID_ARG;
+  if (args->B == 0) return VA_OK;
+  if (!o_part || !lse_part || !aligned(o_part, 16) || !aligned(lse_part, 4))
+    return VA_ERR_INVALID_ARG;
+  const size_t need = va::workspace_layout(*args, S, false).total;
+  if (need && (!args->workspace || !aligned(args->workspace, 256) || args->workspace_bytes < need))
+    return VA_ERR_INVALID_ARG;
+  return va::run_partials(*args, va::SplitRange{S, split_first, split_count}, args->workspace,
+                          o_part, lse_part, (cudaStream_t)stream);
 }
 
 int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, int H,

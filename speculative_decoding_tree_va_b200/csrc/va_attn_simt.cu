@@ -123,7 +123,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
                  const Tkv* __restrict__ c_kv, const Tkv* __restrict__ k_pe, int num_pages,
                  const int32_t* __restrict__ page_table, int max_pages,
                  const int32_t* __restrict__ kv_len_arr, const uint64_t* __restrict__ tree_mask,
-                 int H, int T, float scale_log2, float out_scale, int S, Tout* __restrict__ out,
+                 int H, int T, float scale_log2, float out_scale, int S, int split0,
+                 Tout* __restrict__ out,
                  float* __restrict__ lse_out, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
@@ -143,7 +144,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   const int kv_len = kv_len_arr[b];
   const bool req_ok = kv_len >= T && kv_len <= max_pages * kPage;
   int lo = 0, hi = 0;
-  if (req_ok) split_range(kv_len, S, split, &lo, &hi);
+  if (req_ok) split_range(kv_len, S, split0 + split, &lo, &hi);
   const int P = kv_len - T;
   if (tid == 0) bad_page = 0;
   __syncthreads();
@@ -288,7 +289,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     const float inv = empty ? 0.f : out_scale / l[r];
     const float lse = empty ? -INFINITY : (m[r] + log2f(l[r])) * kLn2;
     const size_t g = (size_t)b * R + row;
-    if (S == 1) {
+    if (!o_part) {
       Tout* o = out + g * kDc + lane * 4;
 #pragma unroll
       for (int gq = 0; gq < 4; ++gq)
@@ -309,27 +310,27 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
 }
 
 template <typename Tq, typename Tkv, typename Tout>
-cudaError_t launch_typed(const va_attn_args& a, int S, float* o_part, float* lse_part,
+cudaError_t launch_typed(const va_attn_args& a, SplitRange sp, float* o_part, float* lse_part,
                          cudaStream_t st) {
   auto kern = attn_simt_kernel<Tq, Tkv, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemTotal);
   if (e != cudaSuccess) return e;
   const int R = a.T * a.H;
-  dim3 grid((R + kRows - 1) / kRows, a.B, S);
+  dim3 grid((R + kRows - 1) / kRows, a.B, sp.count);
   const float kv_scale = (a.flags & VA_FLAG_KV_FP8_E4M3) ? a.kv_scale : 1.f;
   const float scale_log2 = (a.scale * kv_scale) * kLog2e;
   kern<<<grid, kThreads, kSmemTotal, st>>>(
       (const Tq*)a.q_nope, (const Tq*)a.q_pe, (const Tkv*)a.c_kv, (const Tkv*)a.k_pe,
       a.num_pages, a.page_table, a.max_pages, a.kv_len, a.tree_mask, a.H, a.T, scale_log2,
-      kv_scale, S, (Tout*)a.out, a.lse, o_part, lse_part, a.req_status, a.B);
+      kv_scale, sp.S, sp.first, (Tout*)a.out, a.lse, o_part, lse_part, a.req_status, a.B);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                             cudaStream_t st) {
+cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange S, float* o_part,
+                             float* lse_part, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
   const bool fp8 = (a.flags & VA_FLAG_KV_FP8_E4M3) != 0;
   if (a.dtype == VA_F32)

@@ -59,13 +59,15 @@ struct TcParams {
   const void* k_pe;
   const int32_t* page_table;
   const int32_t* kv_len;
+  const int32_t* order;  // grid row y -> request (longest first)
   const uint64_t* tree_mask;
   void* out;
   float* lse;
   float* o_part;
   float* lse_part;
   int32_t* req_status;
-  int B, H, T, R, max_pages, num_pages, S;
+  int B, H, T, R, max_pages, num_pages;
+  int S, split0;  // S-way key partition; grid z = splits split0, split0 + 1, ...
   int stall_mma;  // test hook: issue no tensor-core work (the waits expire)
   float scale_log2;
   float out_scale;  // multiplies the normalised output (an FP8 cache's scale; else 1)
@@ -263,23 +265,46 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
          ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// Request with descending-kv_len rank `y` (ties by index).  Whole-block call.
-__device__ __noinline__ int request_of_rank(const int32_t* kv_len, int B, int y) {
-  __shared__ int found;
-  if (B > 1024) return y;  // large batches keep their natural order
-  if (threadIdx.x == 0) found = y;
-  __syncthreads();
-  for (int i = threadIdx.x; i < B; i += blockDim.x) {
-    const int ki = kv_len[i];
-    int rank = 0;
-    for (int j = 0; j < B; ++j) {
-      const int kj = kv_len[j];
-      rank += (kj > ki) || (kj == ki && j < i);
+// Longest-first order of the requests: order[y] = the request with the y-th
+// largest kv_len, ties by index.  One CTA sorts keys (descending kv_len,
+// ascending index) bitonically in shared memory; batches beyond kMaxSorted
+// keep their natural order (their grids are many waves deep, so the ragged
+// tail that the order shortens is a small share of the launch).
+constexpr int kMaxSorted = 16384;
+constexpr int kOrderThreads = 1024;
+
+__global__ void __launch_bounds__(kOrderThreads)
+request_order_kernel(const int32_t* __restrict__ kv_len, int B, int n, int32_t* __restrict__ order) {
+  extern __shared__ unsigned long long keys[];
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    unsigned long long k = ~0ull;  // padding sorts last
+    if (i < B) {
+      const int v = kv_len[i];
+      const unsigned int len = v < 0 ? 0u : (unsigned int)v;
+      k = ((unsigned long long)(0x7fffffffu - min(len, 0x7fffffffu)) << 32) | (unsigned int)i;
     }
-    if (rank == y) found = i;
+    keys[i] = k;
   }
   __syncthreads();
-  return found;
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const unsigned long long a = keys[i], c = keys[j];
+          if ((a > c) == up) { keys[i] = c; keys[j] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < B; i += blockDim.x) order[i] = (int32_t)(keys[i] & 0xffffffffu);
+}
+
+__global__ void identity_order_kernel(int B, int32_t* __restrict__ order) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B) order[i] = i;
 }
 
 // -------------------------------------------------------------------- kernel
@@ -300,16 +325,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
   const uint32_t rank = cluster_rank();
   // Requests run longest first: grid row y takes the request of rank y in
   // descending kv_len (ties by index), so the ragged tail of the launch is
-  // made of short row tiles.  Every CTA derives the same order itself.
-  const int b = request_of_rank(p.kv_len, p.B, blockIdx.y);
-  const int split = blockIdx.z;
+  // made of short row tiles.
+  const int b = p.order[blockIdx.y];
+  const int split = blockIdx.z;  // position in this launch; the key range is split0 + split
   const int tile_m = blockIdx.x >> 1;
   const int row0 = tile_m * 128 + (int)rank * 64;  // first query row of this CTA
 
   const int kv_len = p.kv_len[b];
   const bool req_ok = kv_len >= p.T && kv_len <= p.max_pages * kPage;
   int lo = 0, hi = 0;
-  if (req_ok) split_range(kv_len, p.S, split, &lo, &hi);
+  if (req_ok) split_range(kv_len, p.S, p.split0 + split, &lo, &hi);
   const int P = kv_len - p.T;
   const int ntiles = hi > lo ? (hi - lo + kTileKeys - 1) / kTileKeys : 0;
 
@@ -651,7 +676,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           const int col = nc * 256 + h * 128 + cc * 32;
           if (!row_in) {
             // nothing to store for rows past the request
-          } else if (p.S == 1) {
+          } else if (!p.o_part) {
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g * kDc + col;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -675,7 +700,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         }
       }
       if (h == 0 && row_in) {
-        if (p.S == 1) p.lse[g] = lse;
+        if (!p.o_part) p.lse[g] = lse;
         else p.lse_part[(size_t)split * rows_total + g] = lse;
       }
     }
@@ -741,8 +766,26 @@ bool encode_2d(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) 
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                           cudaStream_t st, float out_scale) {
+cudaError_t launch_request_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  if (B > kMaxSorted) {
+    identity_order_kernel<<<(B + 255) / 256, 256, 0, st>>>(B, order);
+    return cudaGetLastError();
+  }
+  int n = 1;
+  while (n < B) n <<= 1;
+  const size_t smem = (size_t)n * sizeof(unsigned long long);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(request_order_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  request_order_kernel<<<1, kOrderThreads, smem, st>>>(kv_len, B, n, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc(const va_attn_args& a, SplitRange sp, const int32_t* order,
+                           float* o_part, float* lse_part, cudaStream_t st, float out_scale) {
   if (a.B == 0) return cudaSuccess;
   const long long R = (long long)a.T * a.H;
   const long long rows_total = (long long)a.B * R;
@@ -761,6 +804,7 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   p.k_pe = a.k_pe;
   p.page_table = a.page_table;
   p.kv_len = a.kv_len;
+  p.order = order;
   p.tree_mask = a.tree_mask;
   p.out = a.out;
   p.lse = a.lse;
@@ -773,11 +817,12 @@ cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* l
   p.R = (int)R;
   p.max_pages = a.max_pages;
   p.num_pages = a.num_pages;
-  p.S = S;
+  p.S = sp.S;
+  p.split0 = sp.first;
   p.stall_mma = (a.flags & VA_FLAG_TEST_STALL_MMA) ? 1 : 0;
   p.scale_log2 = a.scale * kLog2e;
   p.out_scale = out_scale;
-  dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)S);
+  dim3 grid((unsigned)(2 * ((R + 127) / 128)), (unsigned)a.B, (unsigned)sp.count);
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tqn, tqp, tckv, tkpe, tckv3, p);
   return cudaGetLastError();
 }

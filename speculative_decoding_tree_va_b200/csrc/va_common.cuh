@@ -52,22 +52,28 @@ inline bool widens_fp8_cache(const va_attn_args& a) {
   return uses_tensor_cores(a) && (a.flags & VA_FLAG_KV_FP8_E4M3);
 }
 
-// Workspace layout of one call: split-KV partials (S > 1), then the widened
-// cache (widens_fp8_cache): bf16 [B * max_pages, 64, 512], bf16
-// [B * max_pages, 64, 64] and an int32 [B, max_pages] page table; every part
+// Workspace layout of one call: on the tensor-core path, the requests'
+// longest-first order (int32 [B]); then the split-KV partials (S > 1 and not
+// a partials-only call, whose partials go to the caller's arrays); then the
+// widened cache (widens_fp8_cache): bf16 [B * max_pages, 64, 512], bf16
+// [B * max_pages, 64, 64] and an int32 [B, max_pages] page table.  Every part
 // starts on a 256-byte boundary.  Offsets are in bytes; `total` is 0 when
 // nothing is needed.
 struct WorkspaceLayout {
-  size_t o_part, lse_part, w_ckv, w_kpe, w_table, total;
+  size_t order, o_part, lse_part, w_ckv, w_kpe, w_table, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S) {
-  WorkspaceLayout w{0, 0, 0, 0, 0, 0};
+inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S, bool partials_here = true) {
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0};
   const size_t rows = (size_t)a.B * a.T * a.H;
   size_t off = 0;
-  if (S > 1) {
+  if (uses_tensor_cores(a)) {
+    w.order = off;
+    off += align256((size_t)a.B * sizeof(int32_t));
+  }
+  if (S > 1 && partials_here) {
     w.o_part = off;
     off += align256((size_t)S * rows * kDc * sizeof(float));
     w.lse_part = off;
@@ -86,6 +92,13 @@ inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S) {
   return w;
 }
 
+// Which splits of the S-way key partition one launch computes: [first,
+// first + count).  Partials go to o_part / lse_part indexed by the split's
+// position in the launch (0 .. count-1).
+struct SplitRange {
+  int S, first, count;
+};
+
 // Launchers implemented in the .cu files (internal C++ linkage).
 cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
                               int budget, int32_t* parents, int32_t* tokens, int32_t* depth,
@@ -95,17 +108,24 @@ cudaError_t launch_tree_accept(const int32_t* parents, const int32_t* tokens,
                                int32_t* accept_len, int32_t* next_token, cudaStream_t st);
 cudaError_t launch_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
                              int32_t* status, cudaStream_t st);
-cudaError_t launch_attn_simt(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                             cudaStream_t st);
+cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange sp, float* o_part,
+                             float* lse_part, cudaStream_t st);
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
                          int out_dtype, void* out, float* lse, cudaStream_t st);
-cudaError_t launch_attn_tc(const va_attn_args& a, int S, float* o_part, float* lse_part,
-                           cudaStream_t st, float out_scale);
+cudaError_t launch_request_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t st);
+cudaError_t launch_attn_tc(const va_attn_args& a, SplitRange sp, const int32_t* order,
+                           float* o_part, float* lse_part, cudaStream_t st, float out_scale);
 cudaError_t launch_kv_widen(const va_attn_args& a, void* w_ckv, void* w_kpe, int32_t* w_table,
                             cudaStream_t st);
 
 // Everything va_verify_attn launches once its arguments are checked and its
 // split count S is known, with the workspace at `ws` laid out as above.
 int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st);
+
+// A partials-only call: splits [first, first + count) of the S-way partition
+// into the caller's o_part / lse_part, no merge; `ws` laid out for
+// (S, partials_here = false).
+int run_partials(const va_attn_args& a, SplitRange sp, void* ws, float* o_part, float* lse_part,
+                 cudaStream_t st);
 
 }  // namespace va

@@ -12,10 +12,12 @@
 //
 // The array has kScratchBytes (VA_NOALLOC_SCRATCH_BYTES) on every device that
 // loads the library, for as long as the process lives.  Every call shares it
-// and it keeps the last call's contents; the split kernels write every partial
-// they later read (empty splits write zeros and -inf), so nothing needs
-// clearing between calls.  Two calls whose work overlaps on the GPU (on
+// and it keeps the last call's contents; every part of the workspace is
+// written before it is read within the call (the request order, the split
+// partials -- empty splits write zeros and -inf -- and the widened pages), so
+// nothing needs clearing between calls.  Two calls whose work overlaps on the GPU (on
 // different streams, or on devices sharing nothing else) race on the array.
+#include <atomic>
 #include <mutex>
 
 #include "va_common.cuh"
@@ -30,22 +32,36 @@ static_assert(kScratchBytes % 256 == 0, "scratch size must keep 256-byte alignme
 static __device__ __align__(256) unsigned char va_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 128;
-void* g_scratch_addr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::atomic<void*> g_scratch_addr[kMaxDevices];  // nullptr until a lookup succeeds
+std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of the scratch array on the current device, looked up with
+// that device current and cached once the lookup has succeeded.  A failed
+// lookup (for instance one attempted during stream capture) is not cached:
+// the call fails with its error, the runtime's last-error state is cleared,
+// and the next call on that device tries again.
 cudaError_t scratch_address(void** addr) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return e;
+  }
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_scratch_once[dev], [dev] {
-    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], va_noalloc_scratch);
-  });
-  if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
-  *addr = g_scratch_addr[dev];
+  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+      e = cudaGetSymbolAddress(&p, va_noalloc_scratch);
+      if (e != cudaSuccess || !p) {
+        (void)cudaGetLastError();
+        return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+      }
+      g_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *addr = p;
   return cudaSuccess;
 }
 

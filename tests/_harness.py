@@ -1,9 +1,14 @@
 """Shared test plumbing: synthetic inputs -> (oracle, CUDA library) -> comparison.
 
 Inputs come from ``speculative_decoding_tree_va_b200.synth``; trees for both
-sides come from the oracle's builder (an oracle input, never a CUDA output).
+sides come from the oracle's builder (an oracle input, never a CUDA output),
+and the oracle derives its visibility mask from those parent pointers itself
+(``oracle_rows``): no value the CUDA library computes ever enters the oracle.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 
@@ -44,10 +49,26 @@ def to_device(inp: synth.Inputs, parents: np.ndarray, device="cuda"):
         dtype=dt)
 
 
-def oracle_rows(inp: synth.Inputs, mask: np.ndarray, rows=None, key_lo=None, key_hi=None):
+def oracle_mask(parents: np.ndarray) -> np.ndarray:
+    """The oracle's own ancestor mask of [B, T] parent pointers (uint64 [B, T, W])."""
+    mask, _ = oracle.ancestor_mask(np.asarray(parents, np.int32))
+    return mask
+
+
+def check_gpu_mask(gpu_mask, parents: np.ndarray, what: str = ""):
+    """The library's mask must equal the oracle's bit for bit."""
+    got = np.ascontiguousarray(np.asarray(gpu_mask)).view(np.uint64)
+    ref = oracle_mask(parents)
+    assert got.shape == ref.shape and np.array_equal(got, ref), f"{what}: tree mask differs"
+
+
+def oracle_rows(inp: synth.Inputs, *, parents: np.ndarray, rows=None, key_lo=None, key_hi=None):
+    """fp64 oracle rows of one workload; the mask comes from ``parents`` through the
+    oracle's own ancestor walk."""
     return oracle.attention_rows(inp.q_nope, inp.q_pe, inp.c_kv, inp.k_pe, inp.page_table,
-                                 inp.kv_len, mask, scale=synth.SCALE, dtype=inp.wl.dtype,
-                                 rows=rows, key_lo=key_lo, key_hi=key_hi, **kv_kwargs(inp))
+                                 inp.kv_len, oracle_mask(parents), scale=synth.SCALE,
+                                 dtype=inp.wl.dtype, rows=rows, key_lo=key_lo, key_hi=key_hi,
+                                 **kv_kwargs(inp))
 
 
 def kv_kwargs(inp: synth.Inputs) -> dict:
@@ -57,10 +78,21 @@ def kv_kwargs(inp: synth.Inputs) -> dict:
     return {}
 
 
+def _log(rec: dict):
+    """Print one parity record; with VA_PARITY_LOG set, also append it as a JSON line."""
+    print("[parity] " + json.dumps(rec))
+    path = os.environ.get("VA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
 def compare(out_gpu, lse_gpu, out_ref, lse_ref, dtype: str, what: str = ""):
     """Element-wise check of (out, lse) rows against the oracle at the dtype's bar.
 
-    -inf lse (absent rows) must match exactly, with an all-zero output."""
+    -inf lse (absent rows) must match exactly, with an all-zero output.  Returns
+    (out max_abs, lse max_abs, elements that needed the bf16 storage allowance)
+    and logs them (``_log``)."""
     out_gpu = np.asarray(out_gpu, np.float64).reshape(out_ref.shape)
     lse_gpu = np.asarray(lse_gpu, np.float64).reshape(lse_ref.shape)
     tol = TOL[dtype]
@@ -76,9 +108,15 @@ def compare(out_gpu, lse_gpu, out_ref, lse_ref, dtype: str, what: str = ""):
         # in bf16 alone costs more (half an ulp = 2^-8 |x| reaches 1e-2 at
         # |x| >= 2.56); there the storage rounding plus 2e-3 is allowed.
         bar = np.maximum(tol["out"], np.abs(out_ref) * 2.0 ** -8 + 2e-3)
+        relaxed = int((err > tol["out"]).sum())
         worst = float((err - bar).max()) if out_ref.size else -1.0
+    else:
+        relaxed, worst = 0, d_out - tol["out"]
+    _log({"what": what, "dtype": dtype, "elements": int(out_ref.size), "out_max_abs": d_out,
+          "lse_max_abs": d_lse, "out_over_plain_bar": relaxed})
+    if dtype == "bf16":
         assert worst <= 0, f"{what}: out max_abs {d_out:.3e} over the bf16 bar"
     else:
-        assert d_out <= tol["out"], f"{what}: out max_abs {d_out:.3e} > {tol['out']}"
+        assert worst <= 0, f"{what}: out max_abs {d_out:.3e} > {tol['out']}"
     assert d_lse <= tol["lse"], f"{what}: lse max_abs {d_lse:.3e} > {tol['lse']}"
-    return d_out, d_lse
+    return d_out, d_lse, relaxed

@@ -27,7 +27,11 @@ int main(void) {
   CHECK(va_workspace_bytes(&a) > 0);
   CHECK(va_verify_attn(&a, 0) == VA_ERR_INVALID_ARG);   /* split without a workspace */
   a.num_splits = 1;
-  CHECK(va_workspace_bytes(&a) == 0);
+  CHECK(va_workspace_bytes(&a) == 256);   /* tensor cores: the request order, int32 [B] */
+  a.dtype = VA_F32;
+  CHECK(va_workspace_bytes(&a) == 0);     /* CUDA cores, one pass: nothing */
+  a.dtype = VA_BF16;
+  CHECK(va_verify_attn_partials(&a, 0, 2, (float*)p, (float*)p, 0) == VA_ERR_INVALID_ARG);
 
   a.T = VA_MAX_QLEN + 1;
   CHECK(va_verify_attn(&a, 0) == VA_ERR_INVALID_ARG);
@@ -56,6 +60,7 @@ int main(void) {
   a.flags |= VA_FLAG_TEST_STALL_MMA;
   CHECK(va_num_splits(&a) == -VA_ERR_INVALID_ARG);
   a.flags = 0;
+  printf("VA_NOALLOC_SCRATCH_BYTES=%lu\n", (unsigned long)VA_NOALLOC_SCRATCH_BYTES);
   printf("host checks ok\n");
   return 0;
 }

@@ -99,14 +99,21 @@ def test_other_host_checks(lib):
 
 
 def test_split_planning_and_workspace(lib):
-    # explicit split count: partials [S,B,T,H,512] f32 + [S,B,T,H] f32, 256-byte aligned
+    # tensor cores: the request order (int32 [B]) first; explicit split count:
+    # partials [S,B,T,H,512] f32 + [S,B,T,H] f32; every part 256-byte aligned
     a = args(num_splits=16)
     rows = 2 * 33 * 64
+    order = 256
     o = (16 * rows * 512 * 4 + 255) // 256 * 256
     l = (16 * rows * 4 + 255) // 256 * 256
     assert lib.va_num_splits(ctypes.byref(a)) == 16
-    assert lib.va_workspace_bytes(ctypes.byref(a)) == o + l
-    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1))) == 0
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == order + o + l
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1))) == order
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, B=300))) == 5 * 256
+    # the CUDA-core kernel needs no order; single pass: no workspace at all
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, dtype=va.VA_F32))) == 0
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, flags=va.VA_FLAG_BF16_CUDA_CORES))) == 0
+    assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=16, dtype=va.VA_F32))) == o + l
     # auto: a big batch needs no split; a long, small batch splits
     assert lib.va_num_splits(ctypes.byref(args(B=64, max_pages=129))) == 1
     s = lib.va_num_splits(ctypes.byref(args(B=4, T=65, max_pages=2050)))
@@ -129,21 +136,45 @@ def test_fp8_cache_split_planning_and_workspace(lib):
     cc = args(B=4, T=65, max_pages=2050, flags=fp8["flags"] | va.VA_FLAG_BF16_CUDA_CORES,
               kv_scale=0.4375)
     assert lib.va_num_splits(ctypes.byref(tc)) != lib.va_num_splits(ctypes.byref(cc))
-    # single pass: only the widened cache (B * max_pages pages) and its page table
+    # single pass: the request order, then the widened cache (B * max_pages
+    # pages) and its page table
     a = args(num_splits=1, **fp8)                     # B = 2, max_pages = 50
     pages = 2 * 50
     up = lambda x: (x + 255) // 256 * 256
     want = up(pages * 64 * 512 * 2) + up(pages * 64 * 64 * 2) + up(pages * 4)
-    assert lib.va_workspace_bytes(ctypes.byref(a)) == want
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == 256 + want
     assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, dtype=va.VA_F32, **fp8))) == 0
-    # with splits the partials come first
+    # with splits the partials come between the order and the widened cache
     a = args(num_splits=4, **fp8)
     rows = 2 * 33 * 64
     parts = up(4 * rows * 512 * 4) + up(4 * rows * 4)
-    assert lib.va_workspace_bytes(ctypes.byref(a)) == parts + want
+    assert lib.va_workspace_bytes(ctypes.byref(a)) == 256 + parts + want
     # the no-allocation entry point refuses, before any launch, what its fixed array cannot hold
     big = args(B=64, max_pages=129, num_splits=1, **fp8)
     assert lib.va_verify_attn_noalloc(ctypes.byref(big), None) == va.VA_ERR_UNSUPPORTED
+
+
+def test_partials_host_checks(lib):
+    """va_verify_attn_partials: explicit partition, split range inside it, its own
+    output arrays; out and lse may be NULL; no launch on any failed check."""
+    f = ctypes.c_void_p(1 << 20)
+    ws = dict(workspace=1 << 24, workspace_bytes=1 << 20)
+    call = lambda a, first, count, o=f, l=f: lib.va_verify_attn_partials(ctypes.byref(a), first,
+                                                                         count, o, l, None)
+    assert call(args(num_splits=0, **ws), 0, 1) == va.VA_ERR_INVALID_ARG     # planned: refused
+    assert call(args(num_splits=8, **ws), -1, 2) == va.VA_ERR_INVALID_ARG
+    assert call(args(num_splits=8, **ws), 7, 2) == va.VA_ERR_INVALID_ARG     # past the last split
+    assert call(args(num_splits=8, **ws), 3, 0) == va.VA_ERR_INVALID_ARG
+    assert call(args(num_splits=8, **ws), 0, 2, o=None) == va.VA_ERR_INVALID_ARG
+    assert call(args(num_splits=8, **ws), 0, 2, o=ctypes.c_void_p((1 << 20) + 4)) == \
+        va.VA_ERR_INVALID_ARG                                                # o_part misaligned
+    assert call(args(num_splits=8), 0, 2) == va.VA_ERR_INVALID_ARG           # no workspace (order)
+    assert call(args(num_splits=8, T=66, **ws), 0, 2) == va.VA_ERR_INVALID_ARG
+    assert call(args(num_splits=8, B=0, out=None, lse=None), 0, 2) == va.VA_OK
+    # its workspace is that of a single-split call: no partials in it
+    a = args(num_splits=8)
+    assert va.partials_workspace_bytes(a) == 256
+    assert va.partials_workspace_bytes(args(num_splits=8, dtype=va.VA_F32)) == 0
 
 
 def test_c99_program_uses_the_host_api(tmp_path):
@@ -158,3 +189,6 @@ def test_c99_program_uses_the_host_api(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "host checks ok" in r.stdout
+    # the binding's copy of the fixed no-allocation array size is the header's
+    m = re.search(r"VA_NOALLOC_SCRATCH_BYTES=(\d+)", r.stdout)
+    assert m and int(m.group(1)) == va.NOALLOC_SCRATCH_BYTES

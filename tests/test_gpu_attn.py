@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from speculative_decoding_tree_va_b200 import synth
-from _harness import compare, oracle_rows, to_device, trees_for
+from _harness import check_gpu_mask, compare, oracle_rows, to_device, trees_for
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,10 @@ def va():
 
 
 def run_gpu(va, inp, parents, path, num_splits=1, rows=None):
-    """Mask + attention on the GPU; returns numpy (out, lse) rows and the mask."""
+    """Mask + attention on the GPU; returns numpy (out, lse) rows and the GPU's mask.
+
+    The mask is returned for a bit-exact check against the oracle's; the oracle
+    never computes with it."""
     import torch
     d = to_device(inp, parents)
     mask, status = va.build_tree_mask(d["parents"])
@@ -51,7 +54,8 @@ def check_full(va, inp, path, num_splits=1, parents=None, what=""):
     if parents is None:
         parents = trees_for(inp)["parent"]
     out, lse, mask = run_gpu(va, inp, parents, path, num_splits)
-    ref_out, ref_lse = oracle_rows(inp, mask)
+    check_gpu_mask(mask, parents, what or inp.wl.name)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents)
     return compare(out, lse, ref_out, ref_lse, inp.wl.dtype, what or inp.wl.name)
 
 
@@ -110,7 +114,8 @@ def test_planner_chosen_splits_match_the_oracle(va, path):
     out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
                               d["kv_len"], mask, scale=synth.SCALE, num_splits=0, flags=flags)
     torch.cuda.synchronize()
-    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64))
+    check_gpu_mask(mask.cpu().numpy(), parents)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents)
     compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
             ref_out, ref_lse, inp.wl.dtype, f"{path}, {S} planned splits")
 
@@ -174,9 +179,10 @@ def test_poisoned_request_stays_contained(va, dtype, path):
     inp.k_pe[inp.page_table[0, 1], 9, 2] = inf_
     parents = trees_for(inp)["parent"]
     out, lse, mask = run_gpu(va, inp, parents, path)
+    check_gpu_mask(mask, parents)
     R = inp.T * inp.wl.H
     rows = np.arange(R, 3 * R, dtype=np.int32)
-    ref_out, ref_lse = oracle_rows(inp, mask, rows=rows)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents, rows=rows)
     compare(out[R:], lse[R:], ref_out, ref_lse, dtype, "requests 1-2")
     assert not np.isfinite(out[:R]).all()   # the poisoned request does see its own inputs
 
@@ -199,10 +205,57 @@ def test_bad_kv_len_and_page_are_flagged(va, dtype, path):
     torch.cuda.synchronize()
     assert st.cpu().tolist() == [0, va.VA_ERR_INVALID_ARG, va.VA_ERR_INVALID_ARG]
     assert torch.isneginf(lse[1:]).all() and not out[1:].float().abs().sum()
-    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64),
+    check_gpu_mask(mask.cpu().numpy(), parents)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents,
                                    rows=np.arange(inp.T * inp.wl.H, dtype=np.int32))
     compare(out[0].float().cpu().numpy().reshape(-1, 512), lse[0].cpu().numpy().reshape(-1),
             ref_out, ref_lse, dtype)
+
+
+# --- partials of split subsets (the per-GPU step of a sharded long prefix) ----
+
+@pytest.mark.parametrize("path", ["f32"] + BF16_PATHS)
+def test_partials_of_split_subsets_match_the_oracle(va, path):
+    """Splits computed in three disjoint groups: each partial equals the oracle's
+    attention over that split's key range, and va_merge over all of them equals
+    the unsplit oracle."""
+    import torch
+    name = "fp32-page-test" if path == "f32" else "bf16-long-prefix"
+    inp = synth.make_inputs(synth.WORKLOADS[name], B=2, H=8, P=(2500, 4000))
+    parents = trees_for(inp)["parent"]
+    d = to_device(inp, parents)
+    mask, _ = va.build_tree_mask(d["parents"])
+    check_gpu_mask(mask.cpu().numpy(), parents)
+    S = 8
+    B, T, H = inp.wl.B, inp.T, inp.wl.H
+    flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
+    args = va.make_args(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
+                        d["kv_len"], mask, torch.empty(0, device="cuda"),
+                        torch.empty(0, device="cuda"), scale=synth.SCALE, num_splits=S,
+                        flags=flags)
+    args.out = args.lse = None                       # not used by a partials-only call
+    need = va.partials_workspace_bytes(args)
+    ws = torch.empty(max(need, 256), device="cuda", dtype=torch.uint8)
+    args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
+    o_all = torch.full((S, B, T, H, 512), float("nan"), device="cuda")
+    l_all = torch.full((S, B, T, H), float("nan"), device="cuda")
+    for first, count in ((0, 3), (3, 1), (4, 4)):
+        va.verify_attn_partials(args, first, count, o_all[first:first + count],
+                                l_all[first:first + count])
+    torch.cuda.synchronize()
+    bounds = synth.split_bounds(inp.kv_len, S)
+    dt = inp.wl.dtype
+    for s in range(S):
+        ref_o, ref_l = oracle_rows(inp, parents=parents, key_lo=bounds[:, s, 0],
+                                   key_hi=bounds[:, s, 1])
+        # partials are fp32 on every path: the bar is the query dtype's
+        compare(o_all[s].cpu().numpy().reshape(-1, 512), l_all[s].cpu().numpy().reshape(-1),
+                ref_o, ref_l, dt, f"{path} partial {s} of {S}")
+    out, lse = va.merge(o_all, l_all, d["dtype"])
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle_rows(inp, parents=parents)
+    compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+            ref_out, ref_lse, dt, f"{path} merged partials")
 
 
 # --- merge ---------------------------------------------------------------------
@@ -228,10 +281,14 @@ def test_merge_against_oracle(va, out_dtype, S):
 # --- full-size workloads on sampled rows ---------------------------------------
 
 FULL = [("bf16-deep", 1), ("bf16-b64-ragged", 1), ("bf16-long-prefix", 16)]
+# the long-prefix workload splits its prefix into 16 to 64 chunks; the wider
+# splits run on the tensor-core path (the CUDA-core path shares the split code)
+FULL_TC_ONLY = [("bf16-long-prefix", 32), ("bf16-long-prefix", 64)]
 
 
-@pytest.mark.parametrize("path", BF16_PATHS)
-@pytest.mark.parametrize("name,S", FULL)
+@pytest.mark.parametrize("path,name,S",
+                         [(p, n, s) for p in BF16_PATHS for n, s in FULL] +
+                         [("tc", n, s) for n, s in FULL_TC_ONLY])
 def test_full_size_sampled_rows(va, path, name, S):
     inp = synth.make_inputs(synth.WORKLOADS[name])
     B, T, H = inp.wl.B, inp.T, inp.wl.H
@@ -240,5 +297,6 @@ def test_full_size_sampled_rows(va, path, name, S):
                              full_request=None if name == "bf16-long-prefix" else 0)
     parents = trees_for(inp)["parent"]
     out, lse, mask = run_gpu(va, inp, parents, path, num_splits=S, rows=rows)
-    ref_out, ref_lse = oracle_rows(inp, mask, rows=rows)
-    compare(out, lse, ref_out, ref_lse, "bf16", name)
+    check_gpu_mask(mask, parents, name)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents, rows=rows)
+    compare(out, lse, ref_out, ref_lse, "bf16", f"{name}, {path}, S={S}")

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 from speculative_decoding_tree_va_b200 import synth
-from _harness import compare, oracle_rows, to_device, trees_for
+from _harness import check_gpu_mask, compare, oracle_rows, to_device, trees_for
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +26,8 @@ def va():
 def test_expired_waits_flag_requests_and_leave_the_context_usable(va):
     import torch
     inp = synth.make_inputs(synth.WORKLOADS["bf16-deep"], B=2, H=16, P=(100, 300), budget=8)
-    d = to_device(inp, trees_for(inp)["parent"])
+    parents = trees_for(inp)["parent"]
+    d = to_device(inp, parents)
     mask, _ = va.build_tree_mask(d["parents"])
     call = dict(scale=synth.SCALE, num_splits=1)
     before = va.device_timeouts()
@@ -44,6 +45,7 @@ def test_expired_waits_flag_requests_and_leave_the_context_usable(va):
                               d["kv_len"], mask, req_status=st, **call)
     torch.cuda.synchronize()
     assert st.cpu().tolist() == [0] * inp.wl.B
-    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64))
+    check_gpu_mask(mask.cpu().numpy(), parents)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents)
     compare(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
             ref_out, ref_lse, "bf16", "after the stalled call")

@@ -48,8 +48,7 @@ def test_c_program_runs_the_step(tmp_path):
     out = np.fromfile(tmp_path / "out.bin", np.uint16).astype(np.uint32) << 16
     out = out.view(np.float32).reshape(-1, synth.D_LATENT)
     lse = np.fromfile(tmp_path / "lse.bin", np.float32)
-    mask, _ = oracle.ancestor_mask(par)
-    ref_out, ref_lse = oracle_rows(inp, mask)
+    ref_out, ref_lse = oracle_rows(inp, parents=par)
     compare(out, lse, ref_out, ref_lse, "bf16", "C program")
     path, alen, nxt = oracle.tree_accept(par, tok, tgt)
     assert np.array_equal(np.fromfile(tmp_path / "path.bin", np.int32).reshape(B, T), path)

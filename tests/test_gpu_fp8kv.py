@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 from speculative_decoding_tree_va_b200 import synth
-from _harness import compare, oracle_rows, to_device, trees_for
+from _harness import check_gpu_mask, compare, oracle_rows, to_device, trees_for
 from test_gpu_attn import check_full, run_gpu
 
 pytestmark = pytest.mark.gpu
@@ -112,7 +112,8 @@ def test_fp8kv_bad_page_is_flagged(va, dtype, path):
     torch.cuda.synchronize()
     assert st.cpu().tolist() == [0, va.VA_ERR_INVALID_ARG]
     assert torch.isneginf(lse[1]).all() and not out[1].float().abs().sum()
-    ref_out, ref_lse = oracle_rows(inp, mask.cpu().numpy().view(np.uint64),
+    check_gpu_mask(mask.cpu().numpy(), parents)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents,
                                    rows=np.arange(inp.T * inp.wl.H, dtype=np.int32))
     compare(out[0].float().cpu().numpy().reshape(-1, 512), lse[0].cpu().numpy().reshape(-1),
             ref_out, ref_lse, dtype)
@@ -149,5 +150,6 @@ def test_full_size_bf16_fp8kv_sampled_rows(va):
     rows = synth.sample_rows(7, B, T, H, 256, full_request=None)
     parents = trees_for(inp)["parent"]
     out, lse, mask = run_gpu(va, inp, parents, "tc", num_splits=inp.wl.splits, rows=rows)
-    ref_out, ref_lse = oracle_rows(inp, mask, rows=rows)
+    check_gpu_mask(mask, parents)
+    ref_out, ref_lse = oracle_rows(inp, parents=parents, rows=rows)
     compare(out, lse, ref_out, ref_lse, "bf16", "bf16-fp8kv-deep")

@@ -111,6 +111,8 @@ def test_greedy_step_in_one_cuda_graph(va):
     path, alen, nxt = torch.empty(B, T, **i32), torch.empty(B, **i32), torch.empty(B, **i32)
     args = va.make_args(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"],
                         d["kv_len"], mask, out, lse, scale=synth.SCALE, num_splits=1)
+    ws = torch.empty(max(va.workspace_bytes(args), 256), device="cuda", dtype=torch.uint8)
+    args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
     P = lambda t: ctypes.c_void_p(t.data_ptr())
 
     def step(stream):
@@ -130,7 +132,7 @@ def test_greedy_step_in_one_cuda_graph(va):
     with torch.cuda.graph(g, stream=side):
         step(side)
     ref_mask, _ = oracle.ancestor_mask(ref_tree["parent"])
-    ref_out, ref_lse = oracle_rows(inp, ref_mask)
+    ref_out, ref_lse = oracle_rows(inp, parents=ref_tree["parent"])
     ref_acc = oracle.tree_accept(ref_tree["parent"], ref_tree["token"], tgt_h)
     for _ in range(2):
         out.zero_()
