@@ -8,11 +8,18 @@
 // so nothing but the running max / sum / output is kept per row.
 //
 // Layout: one CTA = 32 consecutive rows (row = t*H + h) of one request and one
-// key split; 8 warps, warp w owns rows 4w..4w+3.  Key tiles of 32 keys
-// (all 576 q.k dims, fp32 in shared memory, double-buffered with cp.async for
-// fp32 inputs) are shared by the 32 rows.  Scores: lane = key.  Output: lane
-// owns 16 of the 512 latent columns (4 groups of 4, 128 apart) for the
-// warp's 4 rows, so every row's softmax state lives in one warp.
+// key split, 8 warps; key tiles of 16 keys (all 576 q.k dims, fp32 in shared
+// memory, double-buffered; cp.async for fp32 inputs).  Per tile:
+//  * S = Q.K^T (32 x 16): warp w takes dims [72w, 72w + 72) of every row and
+//    key, each lane a 4-row x 4-key register tile (rows i + 8a, keys j + 4b),
+//    so one 16-byte shared load feeds 16 FFMAs; the 8 partial tiles are
+//    summed through shared memory.
+//  * softmax: 8 lanes per row, 2 keys each; the running max moves (and O is
+//    rescaled) only when a tile raises it by more than 2^8.
+//  * O += P.V (32 x 512): warp w owns columns [64w, 64w + 64), each lane an
+//    8-row x 8-column register tile, so two 16-byte loads of P and two of V
+//    feed 64 FFMAs.
+// Row strides of 580 floats keep the strided 16-byte reads conflict-free.
 //
 // FP8 cache: codes are widened to fp32 while they are staged; the cache scale
 // is folded into the score scale and into the output normalisation, so the
@@ -25,13 +32,20 @@ namespace va {
 namespace {
 
 constexpr int kRows = 32;       // rows per CTA
-constexpr int kKeys = 32;       // keys per tile
-constexpr int kThreads = 256;
-constexpr int kQStride = kDqk;       // q rows are read as warp-wide broadcasts
-constexpr int kKStride = kDqk + 4;   // +4 floats: lane-strided float4 reads avoid bank conflicts
-constexpr size_t kSmemQ = (size_t)kRows * kQStride * sizeof(float);
-constexpr size_t kSmemK = (size_t)kKeys * kKStride * sizeof(float);
-constexpr size_t kSmemTotal = kSmemQ + 2 * kSmemK;
+constexpr int kKeys = 16;       // keys per tile
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kStride = kDqk + 4;          // floats per staged Q / K row
+constexpr int kDSlice = kDqk / kWarps;     // q.k dims per warp: 72
+constexpr int kSpStride = 40;              // partial-score tile [key][row], padded
+constexpr int kPStride = kRows + 4;        // probabilities [key][row], padded
+constexpr float kRescaleLog2 = 8.0f;       // lazy max: rescale only past 2^8
+constexpr size_t kSmemQ = (size_t)kRows * kStride * sizeof(float);
+constexpr size_t kSmemK = (size_t)kKeys * kStride * sizeof(float);
+constexpr size_t kSmemSp = (size_t)kWarps * kKeys * kSpStride * sizeof(float);
+constexpr size_t kSmemP = (size_t)kKeys * kPStride * sizeof(float);
+constexpr size_t kSmemTotal = kSmemQ + 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof(float);
+static_assert(kDqk % (4 * kWarps) == 0, "dims split evenly into float4 steps per warp");
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -40,16 +54,6 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n"); }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // Load 16 bytes of `src` (8 bf16 or 4 fp32 values) as fp32 into dst.
 __device__ __forceinline__ void load_row_chunk(float* dst, const float* src) {
@@ -99,7 +103,7 @@ __device__ void stage_keys(float* sK, const Tin* __restrict__ c_kv, const Tin* _
   for (int c = tid; c < kKeys * kChunks; c += kThreads) {
     const int key = c / kChunks;
     const int part = c - key * kChunks;
-    float* dst = sK + key * kKStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+    float* dst = sK + key * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
     const int j = j0 + key;
     if (j < hi && phys >= 0) {
       const size_t krow = (size_t)phys * kPage + (j & (kPage - 1));
@@ -112,6 +116,50 @@ __device__ void stage_keys(float* sK, const Tin* __restrict__ c_kv, const Tin* _
     }
   }
 }
+
+// Key staging for element types that are widened on the way into shared
+// memory (bf16, FP8 codes): the next tile's 16-byte chunks are loaded into
+// registers before the current tile's products and converted and stored after
+// them, so the global loads overlap the arithmetic.  Keys at or past `hi`, and
+// keys of an out-of-range page, become zeros.
+template <typename Tin>
+struct RegStage {
+  static constexpr int V = Elems<Tin>::v;
+  static constexpr int kChunksC = kDc / V, kChunks = kChunksC + kDr / V;
+  static constexpr int kTotal = kKeys * kChunks;
+  static constexpr int kPer = (kTotal + kThreads - 1) / kThreads;
+  uint4 buf[kPer];
+
+  __device__ __forceinline__ void load(const Tin* __restrict__ c_kv, const Tin* __restrict__ k_pe,
+                                       int phys, int j0, int hi, int tid) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int c = tid + i * kThreads;
+      buf[i] = make_uint4(0, 0, 0, 0);
+      if (c < kTotal) {
+        const int key = c / kChunks, part = c - key * kChunks;
+        const int j = j0 + key;
+        if (j < hi && phys >= 0) {
+          const size_t krow = (size_t)phys * kPage + (j & (kPage - 1));
+          const Tin* src = part < kChunksC ? c_kv + krow * kDc + part * V
+                                           : k_pe + krow * kDr + (part - kChunksC) * V;
+          buf[i] = *reinterpret_cast<const uint4*>(src);
+        }
+      }
+    }
+  }
+  __device__ __forceinline__ void store(float* sK, int tid) const {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int c = tid + i * kThreads;
+      if (c < kTotal) {
+        const int key = c / kChunks, part = c - key * kChunks;
+        float* dst = sK + key * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+        load_row_chunk(dst, reinterpret_cast<const Tin*>(&buf[i]));
+      }
+    }
+  }
+};
 
 // Tq: query element type; Tkv: cache element type (Tq, or uint8_t E4M3
 // codes); Tout: output element type.  scale_log2 already holds the cache
@@ -129,8 +177,13 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
   float* sQ = smem;
-  float* sK0 = sQ + kRows * kQStride;
-  float* sK1 = sK0 + kKeys * kKStride;
+  float* sK0 = sQ + kRows * kStride;
+  float* sK1 = sK0 + kKeys * kStride;
+  float* sSp = sK1 + kKeys * kStride;       // [warp][key][row] partial scores
+  float* sP = sSp + kWarps * kKeys * kSpStride;  // [key][row] probabilities
+  float* sAlpha = sP + kKeys * kPStride;    // [row] rescale factor of this tile
+  float* sM = sAlpha + kRows;               // [row] final running max (log2 domain)
+  float* sL = sM + kRows;                   // [row] final sum
   __shared__ int bad_page;
 
   const int tid = threadIdx.x;
@@ -155,7 +208,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     constexpr int kChunksC = kDc / V, kChunks = kChunksC + kDr / V;
     for (int c = tid; c < kRows * kChunks; c += kThreads) {
       const int r = c / kChunks, part = c - r * kChunks;
-      float* dst = sQ + r * kQStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+      float* dst = sQ + r * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
       const int row = row0 + r;
       if (row < R) {
         const size_t g = (size_t)b * R + row;
@@ -169,30 +222,32 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     }
   }
 
-  // Per-row state of this warp's 4 rows (replicated across lanes).
-  float m[4], l[4];
-  uint64_t mw0[4], mw1[4];
-  bool live[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = row0 + warp * 4 + r;
-    m[r] = -INFINITY;
-    l[r] = 0.f;
-    live[r] = false;
-    mw0[r] = mw1[r] = 0;
+  // Softmax role: row sr of the CTA, keys 2*sk and 2*sk + 1 of each tile; the
+  // row's 8 lanes keep identical copies of its running max and sum.
+  const int sr = tid >> 3, sk = tid & 7;
+  float m_used = -INFINITY, l = 0.f;
+  uint64_t mw0 = 0, mw1 = 0;
+  bool live = false;
+  {
+    const int row = row0 + sr;
     if (row < R && req_ok) {
       const int t = row / H;
       const uint64_t* mrow = tree_mask + ((size_t)b * T + t) * W;
-      mw0[r] = mrow[0];
-      mw1[r] = W > 1 ? mrow[1] : 0ull;
-      live[r] = mask_bit(mrow, t);
+      mw0 = mrow[0];
+      mw1 = W > 1 ? mrow[1] : 0ull;
+      live = mask_bit(mrow, t);
     }
   }
-  float acc[4][16];
+  // Q.K^T role: rows qi + 8a, keys qj + 4b, dims [72 warp, +72).
+  const int qi = lane & 7, qj = lane >> 3;
+  // P.V role: rows 8 pi .. 8 pi + 7; columns 64 warp + 4 pj + {0..3} and +32.
+  const int pi = lane >> 3, pj = lane & 7;
+  const int col0 = 64 * warp + 4 * pj;
+  float acc[8][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 16; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
 
   const int ntiles = (hi > lo) ? (hi - lo + kKeys - 1) / kKeys : 0;
   auto phys_of = [&](int j0) -> int {
@@ -200,111 +255,172 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     if (pg < 0 || pg >= num_pages) { bad_page = 1; return -1; }
     return pg;
   };
+  // fp32 keys go to shared memory by cp.async; other types through registers
+  constexpr bool kAsync = sizeof(Tkv) == 4;
+  RegStage<Tkv> reg;
   if (ntiles > 0) stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
   cp_async_commit();
 
   for (int it = 0; it < ntiles; ++it) {
     float* sK = (it & 1) ? sK1 : sK0;
     cp_async_wait_all();
-    __syncthreads();
-    if (it + 1 < ntiles) {
+    __syncthreads();  // tile it staged; the previous tile's P.V is done
+    const bool more = it + 1 < ntiles;
+    if (more) {
       const int jn = lo + (it + 1) * kKeys;
-      stage_keys<Tkv>((it & 1) ? sK0 : sK1, c_kv, k_pe, phys_of(jn), jn, hi, tid);
+      if (kAsync) stage_keys<Tkv>((it & 1) ? sK0 : sK1, c_kv, k_pe, phys_of(jn), jn, hi, tid);
+      else reg.load(c_kv, k_pe, phys_of(jn), jn, hi, tid);
     }
     cp_async_commit();
 
-    // scores: lane = key, 4 rows
-    const int j = lo + it * kKeys + lane;
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- partial scores of this warp's dim slice
     {
-      const float* kr = sK + lane * kKStride;
-      const float* q0 = sQ + (warp * 4) * kQStride;
-#pragma unroll 4
-      for (int d = 0; d < kDqk; d += 4) {
-        const float4 kv = *reinterpret_cast<const float4*>(kr + d);
+      float s[4][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(q0 + r * kQStride + d);
-          s[r] = fmaf(qv.x, kv.x, s[r]);
-          s[r] = fmaf(qv.y, kv.y, s[r]);
-          s[r] = fmaf(qv.z, kv.z, s[r]);
-          s[r] = fmaf(qv.w, kv.w, s[r]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) s[a][c] = 0.f;
+      const float* qb = sQ + qi * kStride + warp * kDSlice;
+      const float* kb = sK + qj * kStride + warp * kDSlice;
+#pragma unroll 3
+      for (int d = 0; d < kDSlice; d += 4) {
+        float4 qv[4], kv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qb + a * 8 * kStride + d);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(kb + c * 4 * kStride + d);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            s[a][c] = fmaf(qv[a].x, kv[c].x, s[a][c]);
+            s[a][c] = fmaf(qv[a].y, kv[c].y, s[a][c]);
+            s[a][c] = fmaf(qv[a].z, kv[c].z, s[a][c]);
+            s[a][c] = fmaf(qv[a].w, kv[c].w, s[a][c]);
+          }
+      }
+      float* sp = sSp + warp * kKeys * kSpStride;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sp[(qj + 4 * c) * kSpStride + qi + 8 * a] = s[a][c];
+    }
+    __syncthreads();  // partial scores visible
+
+    // ---- online softmax of row sr, keys 2 sk, 2 sk + 1
+    {
+      const int jt = lo + it * kKeys;
+      float x[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = 2 * sk + e;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += sSp[(w * kKeys + key) * kSpStride + sr];
+        const int j = jt + key;
+        bool vis = live && j < hi;
+        if (vis && j >= P) {
+          const int i = j - P;
+          vis = ((i < 64 ? (mw0 >> i) : (mw1 >> (i - 64))) & 1ull) != 0;
+        }
+        x[e] = vis ? sum * scale_log2 : -INFINITY;
+      }
+      float tmax = fmaxf(x[0], x[1]);
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+      float alpha = 1.f;
+      if (tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax != -INFINITY)) {
+        alpha = m_used == -INFINITY ? 1.f : exp2f(m_used - tmax);  // O and l are 0 before
+        m_used = tmax;
+      }
+      float p0 = 0.f, p1 = 0.f;
+      if (m_used != -INFINITY) {
+        p0 = exp2f(x[0] - m_used);
+        p1 = exp2f(x[1] - m_used);
+      }
+      float psum = p0 + p1;
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+      l = l * alpha + psum;
+      sP[(2 * sk) * kPStride + sr] = p0;
+      sP[(2 * sk + 1) * kPStride + sr] = p1;
+      if (sk == 0) sAlpha[sr] = alpha;
+    }
+    __syncthreads();  // probabilities and rescale factors visible
+
+    // ---- O += P.V on this lane's 8 x 8 tile
+    {
+      const float4 a0 = *reinterpret_cast<const float4*>(sAlpha + 8 * pi);
+      const float4 a1 = *reinterpret_cast<const float4*>(sAlpha + 8 * pi + 4);
+      const float al[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      bool any = false;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) any |= al[r] != 1.f;
+      if (any) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[r][c] *= al[r];
+      }
+#pragma unroll 4
+      for (int k = 0; k < kKeys; ++k) {
+        const float4 p0 = *reinterpret_cast<const float4*>(sP + k * kPStride + 8 * pi);
+        const float4 p1 = *reinterpret_cast<const float4*>(sP + k * kPStride + 8 * pi + 4);
+        const float4 v0 = *reinterpret_cast<const float4*>(sK + k * kStride + col0);
+        const float4 v1 = *reinterpret_cast<const float4*>(sK + k * kStride + col0 + 32);
+        const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          acc[r][0] = fmaf(pr[r], v0.x, acc[r][0]);
+          acc[r][1] = fmaf(pr[r], v0.y, acc[r][1]);
+          acc[r][2] = fmaf(pr[r], v0.z, acc[r][2]);
+          acc[r][3] = fmaf(pr[r], v0.w, acc[r][3]);
+          acc[r][4] = fmaf(pr[r], v1.x, acc[r][4]);
+          acc[r][5] = fmaf(pr[r], v1.y, acc[r][5]);
+          acc[r][6] = fmaf(pr[r], v1.z, acc[r][6]);
+          acc[r][7] = fmaf(pr[r], v1.w, acc[r][7]);
         }
       }
     }
-    float alpha[4], pk[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      bool vis = live[r] && j < hi;
-      if (vis && j >= P) {
-        const int i = j - P;
-        vis = ((i < 64 ? (mw0[r] >> i) : (mw1[r] >> (i - 64))) & 1ull) != 0;
-      }
-      const float x = vis ? s[r] * scale_log2 : -INFINITY;
-      const float mnew = fmaxf(m[r], warp_max(x));
-      float p = 0.f;
-      alpha[r] = 1.f;
-      if (mnew != -INFINITY) {
-        p = exp2f(x - mnew);
-        alpha[r] = exp2f(m[r] - mnew);  // m = -inf -> 0
-      }
-      l[r] = l[r] * alpha[r] + warp_sum(p);
-      m[r] = mnew;
-      pk[r] = p;
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) acc[r][c] *= alpha[r];
-    // PV: V = the staged c_kv columns; p of key k comes from lane k
-#pragma unroll 4
-    for (int k = 0; k < kKeys; ++k) {
-      float pr[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) pr[r] = __shfl_sync(0xffffffffu, pk[r], k);
-      const float* vr = sK + k * kKStride + lane * 4;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 v = *reinterpret_cast<const float4*>(vr + g * 128);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          acc[r][g * 4 + 0] = fmaf(pr[r], v.x, acc[r][g * 4 + 0]);
-          acc[r][g * 4 + 1] = fmaf(pr[r], v.y, acc[r][g * 4 + 1]);
-          acc[r][g * 4 + 2] = fmaf(pr[r], v.z, acc[r][g * 4 + 2]);
-          acc[r][g * 4 + 3] = fmaf(pr[r], v.w, acc[r][g * 4 + 3]);
-        }
-      }
-    }
+    // the other buffer was last read by the previous tile's P.V, which every
+    // thread finished before this tile's first barrier
+    if (!kAsync && more) reg.store((it & 1) ? sK0 : sK1, tid);
   }
   cp_async_wait_all();
+  if (sk == 0) {
+    sM[sr] = m_used;
+    sL[sr] = l;
+  }
   __syncthreads();
   if (tid == 0 && req_status && (!req_ok || bad_page)) req_status[b] = VA_ERR_INVALID_ARG;
 
-  // epilogue
+  // epilogue: lane writes rows 8 pi + r, columns col0 .. +3 and col0 + 32 .. +3
+  const size_t rows_total = (size_t)B * R;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = row0 + warp * 4 + r;
+  for (int r = 0; r < 8; ++r) {
+    const int rr = 8 * pi + r;
+    const int row = row0 + rr;
     if (row >= R) continue;
-    const bool empty = !(l[r] > 0.f) || !req_ok || bad_page;
-    const float inv = empty ? 0.f : out_scale / l[r];
-    const float lse = empty ? -INFINITY : (m[r] + log2f(l[r])) * kLn2;
+    const float lr = sL[rr];
+    const bool empty = !(lr > 0.f) || !req_ok || bad_page;
+    const float inv = empty ? 0.f : out_scale / lr;
+    const float lse = empty ? -INFINITY : (sM[rr] + log2f(lr)) * kLn2;
     const size_t g = (size_t)b * R + row;
     if (!o_part) {
-      Tout* o = out + g * kDc + lane * 4;
+      Tout* o = out + g * kDc + col0;
 #pragma unroll
-      for (int gq = 0; gq < 4; ++gq)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[gq * 128 + e] = from_f32<Tout>(acc[r][gq * 4 + e] * inv);
-      if (lane == 0) lse_out[g] = lse;
+      for (int e = 0; e < 4; ++e) {
+        o[e] = from_f32<Tout>(acc[r][e] * inv);
+        o[32 + e] = from_f32<Tout>(acc[r][4 + e] * inv);
+      }
+      if (warp == 0 && pj == 0) lse_out[g] = lse;
     } else {
-      const size_t rows_total = (size_t)B * R;
-      float* o = o_part + ((size_t)split * rows_total + g) * kDc + lane * 4;
-#pragma unroll
-      for (int gq = 0; gq < 4; ++gq)
-        *reinterpret_cast<float4*>(o + gq * 128) =
-            make_float4(acc[r][gq * 4 + 0] * inv, acc[r][gq * 4 + 1] * inv,
-                        acc[r][gq * 4 + 2] * inv, acc[r][gq * 4 + 3] * inv);
-      if (lane == 0) lse_part[(size_t)split * rows_total + g] = lse;
+      float* o = o_part + ((size_t)split * rows_total + g) * kDc + col0;
+      *reinterpret_cast<float4*>(o) =
+          make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
+      *reinterpret_cast<float4*>(o + 32) =
+          make_float4(acc[r][4] * inv, acc[r][5] * inv, acc[r][6] * inv, acc[r][7] * inv);
+      if (warp == 0 && pj == 0) lse_part[(size_t)split * rows_total + g] = lse;
     }
   }
 }
