@@ -24,7 +24,10 @@
 //    are addressed out of bounds and read as zeros.
 //  * Warp roles: warp 0 TMA producer, warp 1 MMA issuer (leader CTA only),
 //    warps 2-5 softmax + epilogue.  The MMA order QK(i+1) before PV(i) lets
-//    the softmax of tile i overlap the tensor core.
+//    the softmax of tile i overlap the tensor core.  The producer and MMA
+//    warps wait on barriers with all 32 lanes converged and issue from one
+//    elected lane (a single lane polling in a diverged warp slowed MMA issue
+//    about fourfold).
 //  * Online softmax in the log2 domain.  The running max is only moved (and
 //    O rescaled in TMEM) when a tile raises it by more than 2^8; otherwise
 //    probabilities up to 2^8 go through bf16/fp32 unchanged (exact maths,
@@ -143,6 +146,40 @@ __device__ __noinline__ bool mbar_wait(uint64_t* barp, uint32_t parity, volatile
       return false;
     }
   }
+}
+// Warp-wide bounded wait: every lane of the warp calls it together and gets
+// the same answer.  The producer and the MMA issuer wait like this, with the
+// whole warp converged, and hand the issue to one elected lane: a lone lane
+// that polls barriers in a diverged warp was measured to slow tcgen05.mma
+// issue to ~270 clocks per instruction, against 64 with the warp converged.
+__device__ __noinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int k = 0; k < 32; ++k)
+      if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
+    const bool give_up = __shfl_sync(
+        0xffffffffu, (*abort != 0) || (global_ns() - t0 > kTimeoutNs) ? 1 : 0, 0) != 0;
+    if (give_up) {
+      if ((threadIdx.x & 31) == 0 && !*abort) {
+        *abort = 1;
+        atomicAdd(&g_tc_timeouts, 1u);
+      }
+      __syncwarp();
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool warp_wait(uint64_t* barp, uint32_t parity, volatile int* abort) {
+  const uint32_t bar = smem_u32(barp);
+  if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
+  return warp_wait_slow(bar, parity, abort);
+}
+// One lane of a converged warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n.reg .pred p;\nelect.sync _|p, 0xffffffff;\nselp.u32 %0, 1, 0, p;\n}" : "=r"(e));
+  return e != 0;
 }
 // Last-resort wait used only after an abort (bounded, never marks anything).
 __device__ __noinline__ void mbar_wait_final(uint64_t* barp, uint32_t parity) {
@@ -373,13 +410,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && ntiles > 0) {
-      const uint32_t q_bar = map_to_rank(smem_u32(&c.q_full), 0);
-      if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.q_full), 2 * kQBytes);
-      const int qrow = b * p.R + row0;
-      for (int ch = 0; ch < 8; ++ch)
-        tma_load_2d(smem_u32(sQ + ch * kChunkBytes), &tm_qn, q_bar, ch * 64, qrow);
-      tma_load_2d(smem_u32(sQ + 8 * kChunkBytes), &tm_qp, q_bar, 0, qrow);
+    // The warp walks the slot sequence converged; one elected lane issues.
+    if (ntiles > 0) {
+      if (elect_one()) {
+        const uint32_t q_bar = map_to_rank(smem_u32(&c.q_full), 0);
+        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.q_full), 2 * kQBytes);
+        const int qrow = b * p.R + row0;
+        for (int ch = 0; ch < 8; ++ch)
+          tma_load_2d(smem_u32(sQ + ch * kChunkBytes), &tm_qn, q_bar, ch * 64, qrow);
+        tma_load_2d(smem_u32(sQ + 8 * kChunkBytes), &tm_qp, q_bar, 0, qrow);
+      }
+      __syncwarp();
 
       const int npages_valid = (kv_len + kPage - 1) / kPage;
       const int oob_row = p.num_pages * kPage;  // first row past the pool: zero fill
@@ -392,13 +433,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       int slot = 0;
       uint32_t phase = 0;
       auto advance = [&]() { if (++slot == kRing) { slot = 0; phase ^= 1; } };
-      // wait for the slot, post this slot's TMA bytes; false on abort
-      auto acquire = [&](uint32_t bytes, uint32_t* bar) -> bool {
-        if (!mbar_wait(&c.empty[slot], phase ^ 1, abort)) return false;
-        *bar = map_to_rank(smem_u32(&c.full[slot]), 0);
-        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.full[slot]), 2 * bytes);
-        return true;
-      };
       bool go = true;
       for (int t = 0; t <= ntiles && go; ++t) {
         if (t < ntiles) {  // K chunks: this CTA's two pages of the tile
@@ -406,14 +440,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           const int r0 = page_row(kb / kPage + 2 * (int)rank);
           const int r1 = page_row(kb / kPage + 2 * (int)rank + 1);
           for (int kc = 0; kc < 9 && go; ++kc) {
-            uint32_t bar;
-            go = acquire(kSlotBytes, &bar);
+            go = warp_wait(&c.empty[slot], phase ^ 1, abort);
             if (!go) break;
-            const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
-            const CUtensorMap* map = kc < 8 ? &tm_ckv : &tm_kpe;
-            const int x0 = kc < 8 ? kc * 64 : 0;
-            tma_load_2d(dst, map, bar, x0, r0);
-            tma_load_2d(dst + kChunkBytes, map, bar, x0, r1);
+            if (elect_one()) {
+              const uint32_t bar = map_to_rank(smem_u32(&c.full[slot]), 0);
+              if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.full[slot]), 2 * kSlotBytes);
+              const uint32_t dst = smem_u32(sRing + (size_t)slot * kSlotBytes);
+              const CUtensorMap* map = kc < 8 ? &tm_ckv : &tm_kpe;
+              const int x0 = kc < 8 ? kc * 64 : 0;
+              tma_load_2d(dst, map, bar, x0, r0);
+              tma_load_2d(dst + kChunkBytes, map, bar, x0, r1);
+            }
+            __syncwarp();
             advance();
           }
         }
@@ -424,36 +462,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
             if (k0 >= hi) break;
             const int r = page_row(k0 / kPage);
             for (int nc = 0; nc < 2 && go; ++nc) {
-              uint32_t bar;
-              go = acquire(kSlotBytes, &bar);
+              go = warp_wait(&c.empty[slot], phase ^ 1, abort);
               if (!go) break;
-              tma_load_3d(smem_u32(sRing + (size_t)slot * kSlotBytes), &tm_ckv3, bar, 0, r,
-                          nc * 4 + (int)rank * 2);
+              if (elect_one()) {
+                const uint32_t bar = map_to_rank(smem_u32(&c.full[slot]), 0);
+                if (rank == 0) mbar_arrive_expect_tx(smem_u32(&c.full[slot]), 2 * kSlotBytes);
+                tma_load_3d(smem_u32(sRing + (size_t)slot * kSlotBytes), &tm_ckv3, bar, 0, r,
+                            nc * 4 + (int)rank * 2);
+              }
+              __syncwarp();
               advance();
             }
           }
         }
       }
-      // drain: every slot's last load must be consumed before the CTA may exit
-      for (int s2 = 0; s2 < kRing && go; ++s2) {
-        go = mbar_wait(&c.empty[slot], phase ^ 1, abort);
-        advance();
-      }
-      if (*abort) settle();  // loads already issued land before teardown
-    } else if (lane > 0 && ntiles > 0) {
-      // the other 31 lanes check every page index this split reads
+      // every page index this split reads is checked while the last loads
+      // are consumed (out-of-range pages were read as zeros)
       int bad = 0;
-      for (int pg = lo / kPage + lane - 1; pg < (hi + kPage - 1) / kPage; pg += 31) {
+      for (int pg = lo / kPage + lane; pg < (hi + kPage - 1) / kPage; pg += 32) {
         const int ph = p.page_table[(size_t)b * p.max_pages + pg];
         bad |= (ph < 0 || ph >= p.num_pages);
       }
-      if (bad) c.bad_page = 1;
+      if (__any_sync(0xffffffffu, bad) && lane == 0) c.bad_page = 1;
+      // drain: every slot's last load must be consumed before the CTA may exit
+      for (int s2 = 0; s2 < kRing && go; ++s2) {
+        go = warp_wait(&c.empty[slot], phase ^ 1, abort);
+        advance();
+      }
+      if (*abort) settle();  // loads already issued land before teardown
     }
     __syncwarp();
     named_arrive(2, 160);  // publishes bad_page to the epilogue
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (rank == 0 && lane == 0 && ntiles > 0 && !p.stall_mma) {
+    // The warp walks the slot sequence converged; one elected lane issues
+    // each slot's MMAs and its commit.
+    if (rank == 0 && ntiles > 0 && !p.stall_mma) {
       constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
       const uint32_t sq = smem_u32(sQ), sp = smem_u32(sP), sr = smem_u32(sRing);
       int slot = 0;
@@ -466,52 +510,56 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       const uint64_t dp0 = sw128_desc(sp, 16, 1024);           // P, K-major
       const uint64_t dk0 = sw128_desc(sr, 16, 1024);           // K slot, K-major
       const uint64_t dv0 = sw128_desc(sr, kChunkBytes, 1024);  // V slot, MN-major
-      auto wait = [&](uint64_t* bar, uint32_t par) -> bool {  // fast path inline
-        return mbar_try(smem_u32(bar), par) || mbar_wait(bar, par, abort);
-      };
-      bool ok = wait(&c.q_full, 0);
+      bool ok = warp_wait(&c.q_full, 0, abort);
       auto qk = [&](int t) {
         const uint32_t d = tmem + ((t & 1) ? kTmemS1 : 0);
         for (int kc = 0; kc < 9 && ok; ++kc) {
-          ok = wait(&c.full[slot], phase);
+          ok = warp_wait(&c.full[slot], phase, abort);
           if (!ok) break;
-          tc_fence_after();
-          const uint64_t da = dq0 + (uint64_t)((kc * kChunkBytes) >> 4);
-          const uint64_t db = dk0 + (uint64_t)((slot * kSlotBytes) >> 4);
-          mma_bf16_pair(d, da, db, kIdQK, kc != 0);
-          mma_bf16_pair(d, da + 2, db + 2, kIdQK, 1u);
-          mma_bf16_pair(d, da + 4, db + 4, kIdQK, 1u);
-          mma_bf16_pair(d, da + 6, db + 6, kIdQK, 1u);
-          mma_commit_pair(&c.empty[slot]);
+          if (elect_one()) {
+            tc_fence_after();
+            const uint64_t da = dq0 + (uint64_t)((kc * kChunkBytes) >> 4);
+            const uint64_t db = dk0 + (uint64_t)((slot * kSlotBytes) >> 4);
+            mma_bf16_pair(d, da, db, kIdQK, kc != 0);
+            mma_bf16_pair(d, da + 2, db + 2, kIdQK, 1u);
+            mma_bf16_pair(d, da + 4, db + 4, kIdQK, 1u);
+            mma_bf16_pair(d, da + 6, db + 6, kIdQK, 1u);
+            mma_commit_pair(&c.empty[slot]);
+          }
+          __syncwarp();
           advance();
         }
-        mma_commit_pair(&c.s_full[t & 1]);
+        if (elect_one()) mma_commit_pair(&c.s_full[t & 1]);
+        __syncwarp();
       };
       auto pv = [&](int t) {
         const int kb = lo + t * kTileKeys;
-        if (ok) ok = wait(&c.p_ready, t & 1);
+        if (ok) ok = warp_wait(&c.p_ready, t & 1, abort);
         if (!ok) return;
-        tc_fence_after();
         for (int pg = 0; pg < 4 && ok; ++pg) {
           if (kb + pg * kPage >= hi) break;
           const int nk = min(4, (hi - (kb + pg * kPage) + 15) >> 4);  // 16-key steps in range
           const uint64_t da = dp0 + (uint64_t)((pg * kChunkBytes) >> 4);
           for (int nc = 0; nc < 2 && ok; ++nc) {
-            ok = wait(&c.full[slot], phase);
+            ok = warp_wait(&c.full[slot], phase, abort);
             if (!ok) break;
-            tc_fence_after();
-            const uint32_t d = tmem + kTmemO + nc * 128;
-            const uint64_t db = dv0 + (uint64_t)((slot * kSlotBytes) >> 4);
-            const uint32_t acc0 = (t == 0 && pg == 0) ? 0u : 1u;
-            mma_bf16_pair(d, da, db, kIdPV, acc0);
-            if (nk > 1) mma_bf16_pair(d, da + 2, db + 128, kIdPV, 1u);
-            if (nk > 2) mma_bf16_pair(d, da + 4, db + 256, kIdPV, 1u);
-            if (nk > 3) mma_bf16_pair(d, da + 6, db + 384, kIdPV, 1u);
-            mma_commit_pair(&c.empty[slot]);
+            if (elect_one()) {
+              tc_fence_after();
+              const uint32_t d = tmem + kTmemO + nc * 128;
+              const uint64_t db = dv0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint32_t acc0 = (t == 0 && pg == 0) ? 0u : 1u;
+              mma_bf16_pair(d, da, db, kIdPV, acc0);
+              if (nk > 1) mma_bf16_pair(d, da + 2, db + 128, kIdPV, 1u);
+              if (nk > 2) mma_bf16_pair(d, da + 4, db + 256, kIdPV, 1u);
+              if (nk > 3) mma_bf16_pair(d, da + 6, db + 384, kIdPV, 1u);
+              mma_commit_pair(&c.empty[slot]);
+            }
+            __syncwarp();
             advance();
           }
         }
-        mma_commit_pair(&c.o_done);
+        if (elect_one()) mma_commit_pair(&c.o_done);
+        __syncwarp();
       };
       for (int t = 0; t < ntiles && ok; ++t) {
         qk(t);
@@ -521,7 +569,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       if (!ok) {
         // aborted: issue nothing more, and let every MMA already issued
         // finish before the pair tears down and frees tensor memory
-        mma_commit_pair(&c.mma_drain);
+        if (elect_one()) mma_commit_pair(&c.mma_drain);
+        __syncwarp();
         mbar_wait_final(&c.mma_drain, 0);
       }
     }
