@@ -23,7 +23,7 @@
 //    page-table indexed, one 64-token page per box; pages past the request
 //    are addressed out of bounds and read as zeros.
 //  * Warp roles: warp 0 TMA producer, warp 1 MMA issuer (leader CTA only),
-//    warps 2-5 softmax + epilogue.  The MMA order QK(i+1) before PV(i) lets
+//    warps 2-9 softmax + epilogue.  The MMA order QK(i+1) before PV(i) lets
 //    the softmax of tile i overlap the tensor core.  The producer and MMA
 //    warps wait on barriers with all 32 lanes converged and issue from one
 //    elected lane (a single lane polling in a diverged warp slowed MMA issue
@@ -46,7 +46,8 @@ __device__ unsigned int g_tc_timeouts = 0;  // count of barrier waits that expir
 
 namespace {
 
-constexpr int kThreads = 192;          // 6 warps
+constexpr int kThreads = 320;          // 10 warps: producer, MMA, 8 softmax
+constexpr int kSoftThreads = 256;      // softmax + epilogue warps 2-9
 constexpr int kRing = 7;               // KV ring slots
 constexpr int kSlotBytes = 16384;      // one slot: two 8 KB TMA boxes
 constexpr int kChunkBytes = 8192;      // [64 rows x 64 bf16] swizzled chunk
@@ -87,9 +88,9 @@ struct __align__(16) Ctl {
   uint32_t tmem_base;
   int abort;
   int bad_page;
-  float xmax[2][2][64];  // [tile parity][column half][row]
-  float xsum[2][64];
-  float xsumr[2][64];
+  float xmax[2][4][64];  // [tile parity][key quarter][row]
+  float xsum[4][64];
+  float xsumr[4][64];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kPBytes + (size_t)kRing * kSlotBytes + sizeof(Ctl);
@@ -280,6 +281,12 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 __device__ __forceinline__ void named_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// 2^x (hardware approximation, subnormal results flushed to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -383,7 +390,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     mbar_init(&c.q_full, 1);
     mbar_init(&c.s_full[0], 1);
     mbar_init(&c.s_full[1], 1);
-    mbar_init(&c.p_ready, 8);  // 4 softmax warps x 2 CTAs
+    mbar_init(&c.p_ready, 16);  // 8 softmax warps x 2 CTAs
     mbar_init(&c.o_done, 1);
     mbar_init(&c.mma_drain, 1);
     c.abort = 0;
@@ -492,7 +499,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       if (*abort) settle();  // loads already issued land before teardown
     }
     __syncwarp();
-    named_arrive(2, 160);  // publishes bad_page to the epilogue
+    named_arrive(2, 32 + kSoftThreads);  // publishes bad_page to the epilogue
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The warp walks the slot sequence converged; one elected lane issues
@@ -576,9 +583,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int q = warp & 3;            // TMEM lane quadrant of this warp
+    // Eight warps.  Warp w reads TMEM lane quadrant q = w & 3 (rows
+    // 32 (q & 1) .. +31 of this CTA; key half h = q >> 1 of each tile) and
+    // takes the sub-half sh = (w - 2) >> 2 of it: keys [64 part, +64) of the
+    // tile with part = 2 h + sh.  The four parts of a row combine their maxima
+    // and sums through shared memory.
+    const int q = warp & 3;             // TMEM lane quadrant of this warp
     const int m = 32 * (q & 1) + lane;  // row within the CTA
-    const int h = q >> 1;              // column half: keys [128h, +128) of each tile
+    const int h = q >> 1;               // key half of each tile
+    const int sh = (warp - 2) >> 2;     // sub-half
+    const int part = 2 * h + sh;        // key quarter: also the P chunk and the O columns' half
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int row = row0 + m;
     const bool row_in = row < p.R;
@@ -597,23 +611,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
 
     for (int t = 0; t < ntiles; ++t) {
       const int kb = lo + t * kTileKeys;
-      const int j0 = kb + 128 * h;  // key of this thread's first column
+      const int j0 = kb + 64 * part;  // key of this thread's first column
       mbar_wait(&c.s_full[t & 1], (t >> 1) & 1, abort);
       tc_fence_after();
       __syncwarp();  // tcgen05.ld is warp-collective
-      float x[128];
-      const uint32_t s_addr = tmem + lane_base + ((t & 1) ? kTmemS1 : 0);
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + cc * 32, *reinterpret_cast<float(*)[32]>(&x[cc * 32]));
+      float x[64];
+      const uint32_t s_addr = tmem + lane_base + ((t & 1) ? kTmemS1 : 0) + 64 * sh;
+      tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&x[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
       tmem_wait_ld();
       const bool need_mask = !live || (kb + kTileKeys > P) || (kb + kTileKeys > hi);
       float tmax = -INFINITY;
       if (!need_mask) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) { x[i] *= p.scale_log2; tmax = fmaxf(tmax, x[i]); }
+        for (int i = 0; i < 64; ++i) { x[i] *= p.scale_log2; tmax = fmaxf(tmax, x[i]); }
       } else {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
+        for (int i = 0; i < 64; ++i) {
           const int j = j0 + i;
           bool vis = live && j < hi;
           if (vis && j >= P) {
@@ -624,37 +638,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
           tmax = fmaxf(tmax, x[i]);
         }
       }
-      // combine the two column halves of the row
-      c.xmax[t & 1][h][m] = tmax;
-      named_sync(1, 128);
-      tmax = fmaxf(tmax, c.xmax[t & 1][h ^ 1][m]);
+      // combine the four key quarters of the row
+      c.xmax[t & 1][part][m] = tmax;
+      named_sync(1, kSoftThreads);
+      tmax = fmaxf(fmaxf(c.xmax[t & 1][0][m], c.xmax[t & 1][1][m]),
+                   fmaxf(c.xmax[t & 1][2][m], c.xmax[t & 1][3][m]));
 
       bool rescale = false;
       float alpha = 1.f;
       if (tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax != -INFINITY)) {
         if (m_used != -INFINITY) {
-          alpha = exp2f(m_used - tmax);
+          alpha = ex2(m_used - tmax);
           rescale = true;
         }
         m_used = tmax;
       }
-      uint32_t pk[64];
-      float sum = 0.f, sumr = 0.f;
+      uint32_t pk[32];
+      float sum = 0.f;
       if (m_used == -INFINITY) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) pk[i] = 0u;
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = exp2f(x[2 * i] - m_used);
-          const float p1 = exp2f(x[2 * i + 1] - m_used);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(x[2 * i] - m_used);
+          const float p1 = ex2(x[2 * i + 1] - m_used);
           sum += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
-          sumr += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
         }
       }
-      l = l * alpha + sum;
-      lr = lr * alpha + sumr;
 
       // PV(t-1) must be done before P is overwritten or O rescaled
       if (t > 0) {
@@ -662,12 +674,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         tc_fence_after();
       }
       // tcgen05.ld/st are warp-collective: the whole warp takes this branch
-      // if any of its rows needs it (factor 1 for the others)
+      // if any of its rows needs it (factor 1 for the others).  This warp
+      // rescales the O columns of its sub-half (TMEM chunks 4 sh .. 4 sh + 3).
       __syncwarp();
       if (t > 0 && __any_sync(0xffffffffu, rescale)) {
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 4 * sh; cc < 4 * sh + 4; ++cc) {
           float o[32];
           const uint32_t oa = tmem + lane_base + kTmemO + cc * 32;
           tmem_ld32(oa, o);
@@ -678,19 +691,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
         }
         tmem_wait_st();
       }
-      // P -> shared, K-major 128B-swizzled [64 rows x 64 keys] chunks 2h, 2h+1
+      // P -> shared, K-major 128B-swizzled [64 rows x 64 keys] chunk `part`
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {  // 16 groups of 8 keys
-        const int chunk = 2 * h + (g >> 3);
-        const int k16 = g & 7;  // 16-byte unit within the 128-byte row
-        uint8_t* dst = sP + chunk * kChunkBytes + (m >> 3) * 1024 + (m & 7) * 128 +
+      for (int k16 = 0; k16 < 8; ++k16) {  // 16-byte units of the 128-byte row
+        uint8_t* dst = sP + part * kChunkBytes + (m >> 3) * 1024 + (m & 7) * 128 +
                        ((k16 ^ (m & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pk[4 * k16], pk[4 * k16 + 1], pk[4 * k16 + 2], pk[4 * k16 + 3]);
       }
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(p_ready_leader);
+      // the sum of the rounded probabilities (the normaliser of the output)
+      // is taken after P is handed to the tensor cores, off their path
+      float sumr = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        sumr += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+      l = l * alpha + sum;
+      lr = lr * alpha + sumr;
     }
 
     // ---------------------------------------------------------------- epilogue
@@ -698,12 +718,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
       mbar_wait(&c.o_done, (ntiles - 1) & 1, abort);
       tc_fence_after();
     }
-    c.xsum[h][m] = l;
-    c.xsumr[h][m] = lr;
-    named_sync(1, 128);
-    named_sync(2, 160);
-    const float lsum = l + c.xsum[h ^ 1][m];
-    const float lsumr = lr + c.xsumr[h ^ 1][m];
+    c.xsum[part][m] = l;
+    c.xsumr[part][m] = lr;
+    named_sync(1, kSoftThreads);
+    named_sync(2, 32 + kSoftThreads);
+    const float lsum = (c.xsum[0][m] + c.xsum[1][m]) + (c.xsum[2][m] + c.xsum[3][m]);
+    const float lsumr = (c.xsumr[0][m] + c.xsumr[1][m]) + (c.xsumr[2][m] + c.xsumr[3][m]);
     const bool bad = !req_ok || c.bad_page || *abort;
     const bool empty = bad || !(lsum > 0.f) || !(lsumr > 0.f) || ntiles == 0;
     const float inv = empty ? 0.f : p.out_scale / lsumr;
@@ -711,44 +731,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant_
     __syncwarp();
     {
       // every lane runs the (warp-collective) TMEM loads; only rows inside
-      // the request store
+      // the request store.  This warp writes the latent columns of the O
+      // accumulator sh (nc = sh): [256 sh + 128 h, +128).
       const size_t g = (size_t)b * p.R + (row_in ? row : 0);
       const size_t rows_total = (size_t)p.B * p.R;
-      for (int nc = 0; nc < 2; ++nc) {
+      const int nc = sh;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float o[32];
-          if (ntiles > 0) {
-            tmem_ld32(tmem + lane_base + kTmemO + nc * 128 + cc * 32, o);
-            tmem_wait_ld();
-          }
-          const int col = nc * 256 + h * 128 + cc * 32;
-          if (!row_in) {
-            // nothing to store for rows past the request
-          } else if (!p.o_part) {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g * kDc + col;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 u;
-              u.x = pack_bf16(empty ? 0.f : o[8 * v + 0] * inv, empty ? 0.f : o[8 * v + 1] * inv);
-              u.y = pack_bf16(empty ? 0.f : o[8 * v + 2] * inv, empty ? 0.f : o[8 * v + 3] * inv);
-              u.z = pack_bf16(empty ? 0.f : o[8 * v + 4] * inv, empty ? 0.f : o[8 * v + 5] * inv);
-              u.w = pack_bf16(empty ? 0.f : o[8 * v + 6] * inv, empty ? 0.f : o[8 * v + 7] * inv);
-              reinterpret_cast<uint4*>(dst)[v] = u;
-            }
-          } else {
-            float* dst = p.o_part + ((size_t)split * rows_total + g) * kDc + col;
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              reinterpret_cast<float4*>(dst)[v] =
-                  empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                        : make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
-                                      o[4 * v + 3] * inv);
-          }
-          __syncwarp();  // reconverge before the next warp-collective load
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        if (ntiles > 0) {
+          tmem_ld32(tmem + lane_base + kTmemO + nc * 128 + cc * 32, o);
+          tmem_wait_ld();
         }
+        const int col = nc * 256 + h * 128 + cc * 32;
+        if (!row_in) {
+          // nothing to store for rows past the request
+        } else if (!p.o_part) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g * kDc + col;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16(empty ? 0.f : o[8 * v + 0] * inv, empty ? 0.f : o[8 * v + 1] * inv);
+            u.y = pack_bf16(empty ? 0.f : o[8 * v + 2] * inv, empty ? 0.f : o[8 * v + 3] * inv);
+            u.z = pack_bf16(empty ? 0.f : o[8 * v + 4] * inv, empty ? 0.f : o[8 * v + 5] * inv);
+            u.w = pack_bf16(empty ? 0.f : o[8 * v + 6] * inv, empty ? 0.f : o[8 * v + 7] * inv);
+            reinterpret_cast<uint4*>(dst)[v] = u;
+          }
+        } else {
+          float* dst = p.o_part + ((size_t)split * rows_total + g) * kDc + col;
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            reinterpret_cast<float4*>(dst)[v] =
+                empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                      : make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
+                                    o[4 * v + 3] * inv);
+        }
+        __syncwarp();  // reconverge before the next warp-collective load
       }
-      if (h == 0 && row_in) {
+      if (part == 0 && row_in) {
         if (!p.o_part) p.lse[g] = lse;
         else p.lse_part[(size_t)split * rows_total + g] = lse;
       }
