@@ -849,7 +849,8 @@ cudaError_t launch_request_order(const int32_t* kv_len, int B, int32_t* order, c
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  request_order_kernel<<<1, kOrderThreads, smem, st>>>(kv_len, B, n, order);
+  const int threads = n < kOrderThreads ? (n < 32 ? 32 : n) : kOrderThreads;  // one key per thread
+  request_order_kernel<<<1, threads, smem, st>>>(kv_len, B, n, order);
   return cudaGetLastError();
 }
 
