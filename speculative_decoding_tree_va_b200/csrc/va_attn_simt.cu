@@ -11,9 +11,11 @@
 // key split, 8 warps; key tiles of 16 keys (all 576 q.k dims, fp32 in shared
 // memory, double-buffered; cp.async for fp32 inputs).  Per tile:
 //  * S = Q.K^T (32 x 16): warp w takes dims [72w, 72w + 72) of every row and
-//    key, each lane a 4-row x 4-key register tile (rows i + 8a, keys j + 4b),
-//    so one 16-byte shared load feeds 16 FFMAs; the 8 partial tiles are
-//    summed through shared memory.
+//    key; lane (i, j) keeps the Q of rows i + 8a (a = 0..3) and dims
+//    [72w + 18j, +18) in registers for the whole key range and reads only K
+//    from shared memory (one 8-byte load feeds 8 FFMAs across its 4 rows);
+//    the four dim sub-slices of a warp are summed with shuffles, the 8
+//    warps' partial tiles through shared memory.
 //  * softmax: 8 lanes per row, 2 keys each; the running max moves (and O is
 //    rescaled) only when a tile raises it by more than 2^8.
 //  * O += P.V (32 x 512): warp w owns columns [64w, 64w + 64), each lane an
@@ -37,7 +39,8 @@ constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kStride = kDqk + 4;          // floats per staged Q / K row
 constexpr int kDSlice = kDqk / kWarps;     // q.k dims per warp: 72
-constexpr int kSpStride = 40;              // partial-score tile [key][row], padded
+constexpr int kSub = kDSlice / 4;          // dims per lane (four sub-slices per warp): 18
+constexpr int kSpStride = 36;              // partial-score tile [key][row], padded
 constexpr int kPStride = kRows + 4;        // probabilities [key][row], padded
 constexpr float kRescaleLog2 = 8.0f;       // lazy max: rescale only past 2^8
 constexpr size_t kSmemQ = (size_t)kRows * kStride * sizeof(float);
@@ -45,7 +48,7 @@ constexpr size_t kSmemK = (size_t)kKeys * kStride * sizeof(float);
 constexpr size_t kSmemSp = (size_t)kWarps * kKeys * kSpStride * sizeof(float);
 constexpr size_t kSmemP = (size_t)kKeys * kPStride * sizeof(float);
 constexpr size_t kSmemTotal = kSmemQ + 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof(float);
-static_assert(kDqk % (4 * kWarps) == 0, "dims split evenly into float4 steps per warp");
+static_assert(kDqk % (8 * kWarps) == 0, "dims split evenly into float2 steps per lane");
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -238,7 +241,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
       live = mask_bit(mrow, t);
     }
   }
-  // Q.K^T role: rows qi + 8a, keys qj + 4b, dims [72 warp, +72).
+  // Q.K^T role: rows qi + 8a (a = 0..3), dims [72 warp + 18 qj, +18), all keys.
   const int qi = lane & 7, qj = lane >> 3;
   // P.V role: rows 8 pi .. 8 pi + 7; columns 64 warp + 4 pj + {0..3} and +32.
   const int pi = lane >> 3, pj = lane & 7;
@@ -260,6 +263,22 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   RegStage<Tkv> reg;
   if (ntiles > 0) stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
   cp_async_commit();
+  // this lane's Q: rows qi + 8 a, dims [72 warp + 18 qj, +18), kept in
+  // registers for every key tile
+  float qr[4][kSub];
+  cp_async_wait_all();
+  __syncthreads();
+  {
+    const float* qb = sQ + qi * kStride + warp * kDSlice + kSub * qj;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int m2 = 0; m2 < kSub / 2; ++m2) {
+        const float2 v = *reinterpret_cast<const float2*>(qb + a * 8 * kStride + 2 * m2);
+        qr[a][2 * m2] = v.x;
+        qr[a][2 * m2 + 1] = v.y;
+      }
+  }
 
   for (int it = 0; it < ntiles; ++it) {
     float* sK = (it & 1) ? sK1 : sK0;
@@ -273,37 +292,56 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     }
     cp_async_commit();
 
-    // ---- partial scores of this warp's dim slice
+    // ---- partial scores of this warp's dim slice: the lane's Q rows stay in
+    // registers (qr), only K comes from shared memory; the warp's four dim
+    // sub-slices are summed with shuffles before the cross-warp reduction
     {
-      float s[4][4];
+      const bool b0 = (qj & 1) != 0, b1 = (qj >> 1) != 0;
+      float* sp = sSp + warp * kKeys * kSpStride;
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int half = 0; half < 2; ++half) {
+        float acc8[4][8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) s[a][c] = 0.f;
-      const float* qb = sQ + qi * kStride + warp * kDSlice;
-      const float* kb = sK + qj * kStride + warp * kDSlice;
-#pragma unroll 3
-      for (int d = 0; d < kDSlice; d += 4) {
-        float4 qv[4], kv[4];
+        for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qb + a * 8 * kStride + d);
+          for (int c = 0; c < 8; ++c) acc8[a][c] = 0.f;
+        const float* kb = sK + (8 * half) * kStride + warp * kDSlice + kSub * qj;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(kb + c * 4 * kStride + d);
+        for (int c = 0; c < 8; ++c) {
+          float kv[kSub];
+#pragma unroll
+          for (int m2 = 0; m2 < kSub / 2; ++m2) {
+            const float2 v = *reinterpret_cast<const float2*>(kb + c * kStride + 2 * m2);
+            kv[2 * m2] = v.x;
+            kv[2 * m2 + 1] = v.y;
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int d = 0; d < kSub; ++d) acc8[a][c] = fmaf(qr[a][d], kv[d], acc8[a][c]);
+        }
+        // lanes qi + 8 qj, qj = 0..3, hold the same rows and keys over four
+        // dim sub-slices: halve the keys per lane twice while summing pairs
+        float r1[4][4];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            s[a][c] = fmaf(qv[a].x, kv[c].x, s[a][c]);
-            s[a][c] = fmaf(qv[a].y, kv[c].y, s[a][c]);
-            s[a][c] = fmaf(qv[a].z, kv[c].z, s[a][c]);
-            s[a][c] = fmaf(qv[a].w, kv[c].w, s[a][c]);
+            const float mine = b0 ? acc8[a][4 + c] : acc8[a][c];
+            const float give = b0 ? acc8[a][c] : acc8[a][4 + c];
+            r1[a][c] = mine + __shfl_xor_sync(0xffffffffu, give, 8);
+          }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float mine = b1 ? r1[a][2 + c] : r1[a][c];
+            const float give = b1 ? r1[a][c] : r1[a][2 + c];
+            const float v = mine + __shfl_xor_sync(0xffffffffu, give, 16);
+            // keys 8 half + 4 b0 + 2 b1 + c of row qi + 8 a, over the warp's dims
+            sp[(8 * half + 4 * b0 + 2 * b1 + c) * kSpStride + qi + 8 * a] = v;
           }
       }
-      float* sp = sSp + warp * kKeys * kSpStride;
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) sp[(qj + 4 * c) * kSpStride + qi + 8 * a] = s[a][c];
     }
     __syncthreads();  // partial scores visible
 
