@@ -90,6 +90,18 @@ __device__ __forceinline__ void load_row_chunk(float* dst, const uint8_t* src) {
   }
 }
 
+// Two fp32 fused multiply-adds in one instruction (sm_100 packed f32x2),
+// each rounded to nearest exactly like fmaf: d = a * b + c per element.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
 template <typename Tin>
 struct Elems {  // values per 16-byte chunk
   static constexpr int v = 16 / sizeof(Tin);
@@ -246,11 +258,11 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   // P.V role: rows 8 pi .. 8 pi + 7; columns 64 warp + 4 pj + {0..3} and +32.
   const int pi = lane >> 3, pj = lane & 7;
   const int col0 = 64 * warp + 4 * pj;
-  float acc[8][8];
+  float2 acc[8][4];  // columns (col0 + 2c, +1) for c < 2, (col0 + 32 + 2(c-2), +1) after
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < 4; ++c) acc[r][c] = make_float2(0.f, 0.f);
 
   const int ntiles = (hi > lo) ? (hi - lo + kKeys - 1) / kKeys : 0;
   auto phys_of = [&](int j0) -> int {
@@ -265,7 +277,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   cp_async_commit();
   // this lane's Q: rows qi + 8 a, dims [72 warp + 18 qj, +18), kept in
   // registers for every key tile
-  float qr[4][kSub];
+  float2 qr[4][kSub / 2];  // (even dim, odd dim) pairs
   cp_async_wait_all();
   __syncthreads();
   {
@@ -273,11 +285,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int m2 = 0; m2 < kSub / 2; ++m2) {
-        const float2 v = *reinterpret_cast<const float2*>(qb + a * 8 * kStride + 2 * m2);
-        qr[a][2 * m2] = v.x;
-        qr[a][2 * m2 + 1] = v.y;
-      }
+      for (int m2 = 0; m2 < kSub / 2; ++m2)
+        qr[a][m2] = *reinterpret_cast<const float2*>(qb + a * 8 * kStride + 2 * m2);
   }
 
   for (int it = 0; it < ntiles; ++it) {
@@ -300,26 +309,29 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
       float* sp = sSp + warp * kKeys * kSpStride;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        // even and odd dims accumulate in the two halves of a packed pair
+        float2 acc2[4][8];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc2[a][c] = make_float2(0.f, 0.f);
+        const float* kb = sK + (8 * half) * kStride + warp * kDSlice + kSub * qj;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float2 kv[kSub / 2];
+#pragma unroll
+          for (int m2 = 0; m2 < kSub / 2; ++m2)
+            kv[m2] = *reinterpret_cast<const float2*>(kb + c * kStride + 2 * m2);
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int m2 = 0; m2 < kSub / 2; ++m2) acc2[a][c] = fma2(qr[a][m2], kv[m2], acc2[a][c]);
+        }
         float acc8[4][8];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) acc8[a][c] = 0.f;
-        const float* kb = sK + (8 * half) * kStride + warp * kDSlice + kSub * qj;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float kv[kSub];
-#pragma unroll
-          for (int m2 = 0; m2 < kSub / 2; ++m2) {
-            const float2 v = *reinterpret_cast<const float2*>(kb + c * kStride + 2 * m2);
-            kv[2 * m2] = v.x;
-            kv[2 * m2 + 1] = v.y;
-          }
-#pragma unroll
-          for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int d = 0; d < kSub; ++d) acc8[a][c] = fmaf(qr[a][d], kv[d], acc8[a][c]);
-        }
+          for (int c = 0; c < 8; ++c) acc8[a][c] = acc2[a][c].x + acc2[a][c].y;
         // lanes qi + 8 qj, qj = 0..3, hold the same rows and keys over four
         // dim sub-slices: halve the keys per lane twice while summing pairs
         float r1[4][4];
@@ -398,7 +410,10 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) acc[r][c] *= al[r];
+          for (int c = 0; c < 4; ++c) {
+            acc[r][c].x *= al[r];
+            acc[r][c].y *= al[r];
+          }
       }
 #pragma unroll 4
       for (int k = 0; k < kKeys; ++k) {
@@ -407,16 +422,13 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         const float4 v0 = *reinterpret_cast<const float4*>(sK + k * kStride + col0);
         const float4 v1 = *reinterpret_cast<const float4*>(sK + k * kStride + col0 + 32);
         const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        const float2 vv[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w),
+                              make_float2(v1.x, v1.y), make_float2(v1.z, v1.w)};
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          acc[r][0] = fmaf(pr[r], v0.x, acc[r][0]);
-          acc[r][1] = fmaf(pr[r], v0.y, acc[r][1]);
-          acc[r][2] = fmaf(pr[r], v0.z, acc[r][2]);
-          acc[r][3] = fmaf(pr[r], v0.w, acc[r][3]);
-          acc[r][4] = fmaf(pr[r], v1.x, acc[r][4]);
-          acc[r][5] = fmaf(pr[r], v1.y, acc[r][5]);
-          acc[r][6] = fmaf(pr[r], v1.z, acc[r][6]);
-          acc[r][7] = fmaf(pr[r], v1.w, acc[r][7]);
+          const float2 pp = make_float2(pr[r], pr[r]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fma2(pp, vv[c], acc[r][c]);
         }
       }
     }
@@ -447,17 +459,19 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     if (!o_part) {
       Tout* o = out + g * kDc + col0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        o[e] = from_f32<Tout>(acc[r][e] * inv);
-        o[32 + e] = from_f32<Tout>(acc[r][4 + e] * inv);
+      for (int e = 0; e < 2; ++e) {
+        o[2 * e] = from_f32<Tout>(acc[r][e].x * inv);
+        o[2 * e + 1] = from_f32<Tout>(acc[r][e].y * inv);
+        o[32 + 2 * e] = from_f32<Tout>(acc[r][2 + e].x * inv);
+        o[32 + 2 * e + 1] = from_f32<Tout>(acc[r][2 + e].y * inv);
       }
       if (warp == 0 && pj == 0) lse_out[g] = lse;
     } else {
       float* o = o_part + ((size_t)split * rows_total + g) * kDc + col0;
-      *reinterpret_cast<float4*>(o) =
-          make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
-      *reinterpret_cast<float4*>(o + 32) =
-          make_float4(acc[r][4] * inv, acc[r][5] * inv, acc[r][6] * inv, acc[r][7] * inv);
+      *reinterpret_cast<float4*>(o) = make_float4(acc[r][0].x * inv, acc[r][0].y * inv,
+                                                  acc[r][1].x * inv, acc[r][1].y * inv);
+      *reinterpret_cast<float4*>(o + 32) = make_float4(acc[r][2].x * inv, acc[r][2].y * inv,
+                                                       acc[r][3].x * inv, acc[r][3].y * inv);
       if (warp == 0 && pj == 0) lse_part[(size_t)split * rows_total + g] = lse;
     }
   }
