@@ -230,9 +230,11 @@ int va_num_splits(const va_attn_args* args);
  *   s_j = scale * (q_nope . c_kv_j + q_pe . k_pe_j)
  *   out = sum_j softmax(s)_j c_kv_j      lse = ln sum_j exp(s_j)
  * A row whose own tree bit is clear (absent node) gets out = 0, lse = -inf.
- * With S > 1 splits, split s covers keys [s*C, min((s+1)*C, kv_len)) with
- * C = ceil(ceil(kv_len / S) / 256) * 256; the partials go to the workspace
- * and va_merge combines them on the same stream.
+ * With S > 1 splits, split s covers keys [e(s), e(s+1)): e(0) = 0,
+ * e(S) = kv_len, and for 0 < s < S, e(s) = min(kv_len, 256 * floor((2 s kv_len
+ * + 256 S) / (512 S))), i.e. s * kv_len / S rounded to the nearest multiple
+ * of 256, ties up (splits may be empty when kv_len < 128 S); the partials go
+ * to the workspace and va_merge combines them on the same stream.
  * bf16 runs on tensor cores with fp32 accumulation; fp32, and any call with
  * an FP8 cache (VA_FLAG_KV_FP8_E4M3), on CUDA cores.
  * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, 0 <= B <= VA_MAX_BATCH

@@ -8,15 +8,16 @@
 // so nothing but the running max / sum / output is kept per row.
 //
 // Layout: one CTA = 32 consecutive rows (row = t*H + h) of one request and one
-// key split, 8 warps; key tiles of 16 keys (all 576 q.k dims, fp32 in shared
-// memory, double-buffered; cp.async for fp32 inputs).  Per tile:
+// key split, 8 warps; key tiles of 32 keys (all 576 q.k dims, fp32 in shared
+// memory, double-buffered; cp.async for fp32 inputs; the staged Q shares the
+// second key buffer, which is free until the second tile).  Per tile:
 //  * S = Q.K^T (32 x 16): warp w takes dims [72w, 72w + 72) of every row and
 //    key; lane (i, j) keeps the Q of rows i + 8a (a = 0..3) and dims
 //    [72w + 18j, +18) in registers for the whole key range and reads only K
 //    from shared memory (one 8-byte load feeds 8 FFMAs across its 4 rows);
 //    the four dim sub-slices of a warp are summed with shuffles, the 8
 //    warps' partial tiles through shared memory.
-//  * softmax: 8 lanes per row, 2 keys each; the running max moves (and O is
+//  * softmax: 8 lanes per row, 4 keys each; the running max moves (and O is
 //    rescaled) only when a tile raises it by more than 2^8.
 //  * O += P.V (32 x 512): warp w owns columns [64w, 64w + 64), each lane an
 //    8-row x 8-column register tile, so two 16-byte loads of P and two of V
@@ -34,7 +35,7 @@ namespace va {
 namespace {
 
 constexpr int kRows = 32;       // rows per CTA
-constexpr int kKeys = 16;       // keys per tile
+constexpr int kKeys = 32;       // keys per tile
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kStride = kDqk + 4;          // floats per staged Q / K row
@@ -43,12 +44,13 @@ constexpr int kSub = kDSlice / 4;          // dims per lane (four sub-slices per
 constexpr int kSpStride = 36;              // partial-score tile [key][row], padded
 constexpr int kPStride = kRows + 4;        // probabilities [key][row], padded
 constexpr float kRescaleLog2 = 8.0f;       // lazy max: rescale only past 2^8
-constexpr size_t kSmemQ = (size_t)kRows * kStride * sizeof(float);
 constexpr size_t kSmemK = (size_t)kKeys * kStride * sizeof(float);
 constexpr size_t kSmemSp = (size_t)kWarps * kKeys * kSpStride * sizeof(float);
 constexpr size_t kSmemP = (size_t)kKeys * kPStride * sizeof(float);
-constexpr size_t kSmemTotal = kSmemQ + 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof(float);
+constexpr size_t kSmemTotal = 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof(float);
 static_assert(kDqk % (8 * kWarps) == 0, "dims split evenly into float2 steps per lane");
+static_assert(kRows <= kKeys, "the staged Q fits in a key buffer");
+static_assert(kKeys % 8 == 0 && kKeys / 8 <= 8, "8-key groups in Q.K^T; 8 softmax lanes per row");
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -134,24 +136,27 @@ __device__ void stage_keys(float* sK, const Tin* __restrict__ c_kv, const Tin* _
 
 // Key staging for element types that are widened on the way into shared
 // memory (bf16, FP8 codes): the next tile's 16-byte chunks are loaded into
-// registers before the current tile's products and converted and stored after
-// them, so the global loads overlap the arithmetic.  Keys at or past `hi`, and
-// keys of an out-of-range page, become zeros.
+// registers in two halves, one before the current tile's Q.K^T and one before
+// its P.V, and each half is converted and stored after the products it
+// overlaps.  Keys at or past `hi`, and keys of an out-of-range page, become
+// zeros.
 template <typename Tin>
 struct RegStage {
   static constexpr int V = Elems<Tin>::v;
   static constexpr int kChunksC = kDc / V, kChunks = kChunksC + kDr / V;
   static constexpr int kTotal = kKeys * kChunks;
-  static constexpr int kPer = (kTotal + kThreads - 1) / kThreads;
+  static constexpr int kPer = (kTotal / 2 + kThreads - 1) / kThreads;  // per half
+  static_assert(kTotal % 2 == 0, "halves of equal size");
   uint4 buf[kPer];
 
+  // half h covers chunks [h kTotal/2, (h + 1) kTotal/2)
   __device__ __forceinline__ void load(const Tin* __restrict__ c_kv, const Tin* __restrict__ k_pe,
-                                       int phys, int j0, int hi, int tid) {
+                                       int phys, int j0, int hi, int tid, int h) {
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int c = tid + i * kThreads;
+      const int c = h * (kTotal / 2) + tid + i * kThreads;
       buf[i] = make_uint4(0, 0, 0, 0);
-      if (c < kTotal) {
+      if (c < (h + 1) * (kTotal / 2)) {
         const int key = c / kChunks, part = c - key * kChunks;
         const int j = j0 + key;
         if (j < hi && phys >= 0) {
@@ -163,11 +168,11 @@ struct RegStage {
       }
     }
   }
-  __device__ __forceinline__ void store(float* sK, int tid) const {
+  __device__ __forceinline__ void store(float* sK, int tid, int h) const {
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int c = tid + i * kThreads;
-      if (c < kTotal) {
+      const int c = h * (kTotal / 2) + tid + i * kThreads;
+      if (c < (h + 1) * (kTotal / 2)) {
         const int key = c / kChunks, part = c - key * kChunks;
         float* dst = sK + key * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
         load_row_chunk(dst, reinterpret_cast<const Tin*>(&buf[i]));
@@ -191,9 +196,9 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
                  float* __restrict__ lse_out, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
-  float* sQ = smem;
-  float* sK0 = sQ + kRows * kStride;
-  float* sK1 = sK0 + kKeys * kStride;
+  float* sK0 = smem;
+  float* sK1 = sK0 + kKeys * kStride;       // also the staged Q until tile 1 is staged
+  float* sQ = sK1;
   float* sSp = sK1 + kKeys * kStride;       // [warp][key][row] partial scores
   float* sP = sSp + kWarps * kKeys * kSpStride;  // [key][row] probabilities
   float* sAlpha = sP + kKeys * kPStride;    // [row] rescale factor of this tile
@@ -237,8 +242,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     }
   }
 
-  // Softmax role: row sr of the CTA, keys 2*sk and 2*sk + 1 of each tile; the
-  // row's 8 lanes keep identical copies of its running max and sum.
+  // Softmax role: row sr of the CTA, keys sk + 8 e (e = 0..3) of each tile;
+  // the row's 8 lanes keep identical copies of its running max and sum.
   const int sr = tid >> 3, sk = tid & 7;
   float m_used = -INFINITY, l = 0.f;
   uint64_t mw0 = 0, mw1 = 0;
@@ -291,13 +296,16 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
 
   for (int it = 0; it < ntiles; ++it) {
     float* sK = (it & 1) ? sK1 : sK0;
+    float* sKn = (it & 1) ? sK0 : sK1;
     cp_async_wait_all();
-    __syncthreads();  // tile it staged; the previous tile's P.V is done
+    __syncthreads();  // tile it staged; the previous tile's P.V (and, at the
+                      // first tile, every read of the staged Q) is done
     const bool more = it + 1 < ntiles;
+    const int jn = lo + (it + 1) * kKeys;
+    const int physn = more ? phys_of(jn) : -1;
     if (more) {
-      const int jn = lo + (it + 1) * kKeys;
-      if (kAsync) stage_keys<Tkv>((it & 1) ? sK0 : sK1, c_kv, k_pe, phys_of(jn), jn, hi, tid);
-      else reg.load(c_kv, k_pe, phys_of(jn), jn, hi, tid);
+      if (kAsync) stage_keys<Tkv>(sKn, c_kv, k_pe, physn, jn, hi, tid);
+      else reg.load(c_kv, k_pe, physn, jn, hi, tid, 0);
     }
     cp_async_commit();
 
@@ -308,7 +316,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
       const bool b0 = (qj & 1) != 0, b1 = (qj >> 1) != 0;
       float* sp = sSp + warp * kKeys * kSpStride;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < kKeys / 8; ++half) {
         // even and odd dims accumulate in the two halves of a packed pair
         float2 acc2[4][8];
 #pragma unroll
@@ -355,15 +363,22 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
           }
       }
     }
+    // the other buffer is free (see the top of the loop): the first half of
+    // the next tile goes in, the second half's loads overlap P.V
+    if (!kAsync && more) {
+      reg.store(sKn, tid, 0);
+      reg.load(c_kv, k_pe, physn, jn, hi, tid, 1);
+    }
     __syncthreads();  // partial scores visible
 
-    // ---- online softmax of row sr, keys 2 sk, 2 sk + 1
+    // ---- online softmax of row sr, keys sk + 8 e
     {
+      constexpr int kE = kKeys / 8;
       const int jt = lo + it * kKeys;
-      float x[2];
+      float x[kE];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int key = 2 * sk + e;
+      for (int e = 0; e < kE; ++e) {
+        const int key = sk + 8 * e;
         float sum = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) sum += sSp[(w * kKeys + key) * kSpStride + sr];
@@ -375,7 +390,9 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         }
         x[e] = vis ? sum * scale_log2 : -INFINITY;
       }
-      float tmax = fmaxf(x[0], x[1]);
+      float tmax = x[0];
+#pragma unroll
+      for (int e = 1; e < kE; ++e) tmax = fmaxf(tmax, x[e]);
 #pragma unroll
       for (int o = 4; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
       float alpha = 1.f;
@@ -383,17 +400,16 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         alpha = m_used == -INFINITY ? 1.f : exp2f(m_used - tmax);  // O and l are 0 before
         m_used = tmax;
       }
-      float p0 = 0.f, p1 = 0.f;
-      if (m_used != -INFINITY) {
-        p0 = exp2f(x[0] - m_used);
-        p1 = exp2f(x[1] - m_used);
+      float psum = 0.f;
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        const float p = m_used != -INFINITY ? exp2f(x[e] - m_used) : 0.f;
+        psum += p;
+        sP[(sk + 8 * e) * kPStride + sr] = p;
       }
-      float psum = p0 + p1;
 #pragma unroll
       for (int o = 4; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
       l = l * alpha + psum;
-      sP[(2 * sk) * kPStride + sr] = p0;
-      sP[(2 * sk + 1) * kPStride + sr] = p1;
       if (sk == 0) sAlpha[sr] = alpha;
     }
     __syncthreads();  // probabilities and rescale factors visible
@@ -432,9 +448,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         }
       }
     }
-    // the other buffer was last read by the previous tile's P.V, which every
-    // thread finished before this tile's first barrier
-    if (!kAsync && more) reg.store((it & 1) ? sK0 : sK1, tid);
+    if (!kAsync && more) reg.store(sKn, tid, 1);
   }
   cp_async_wait_all();
   if (sk == 0) {

@@ -30,14 +30,19 @@ __device__ __forceinline__ bool mask_bit(const uint64_t* row, int i) {
   return (row[i >> 6] >> (i & 63)) & 1ull;
 }
 
-// Split-KV chunk bounds, as fixed in the public header:
-// C = ceil(ceil(kv_len / S) / 256) * 256, split s = [s*C, min((s+1)*C, kv_len)).
+// Split-KV partition, as fixed in the public header: split s covers
+// [e(s), e(s+1)), where e(0) = 0, e(S) = kv_len and, in between, e(s) is
+// s * kv_len / S rounded to the nearest multiple of 256 (ties up), at most
+// kv_len.  Every split's length is within 256 keys of kv_len / S.
+__host__ __device__ __forceinline__ int split_edge(int kv_len, int S, int s) {
+  if (s >= S) return kv_len;
+  const long long A = VA_SPLIT_ALIGN;
+  const long long e = (2LL * s * kv_len + S * A) / (2LL * S * A) * A;
+  return (int)(e < kv_len ? e : kv_len);
+}
 __host__ __device__ __forceinline__ void split_range(int kv_len, int S, int s, int* lo, int* hi) {
-  int per = (kv_len + S - 1) / S;
-  int chunk = (per + VA_SPLIT_ALIGN - 1) / VA_SPLIT_ALIGN * VA_SPLIT_ALIGN;
-  long long a = (long long)s * chunk, b = (long long)(s + 1) * chunk;
-  *lo = (int)(a < kv_len ? a : kv_len);
-  *hi = (int)(b < kv_len ? b : kv_len);
+  *lo = split_edge(kv_len, S, s);
+  *hi = split_edge(kv_len, S, s + 1);
 }
 
 // The kernel a va_verify_attn call runs on: bf16 queries go to the tensor

@@ -248,13 +248,17 @@ def sample_rows(rng_seed: int, B: int, T: int, H: int, n: int,
 
 def split_bounds(kv_len: np.ndarray, splits: int, align: int = 256) -> np.ndarray:
     """Key ranges [lo, hi) of the flash-decode split, as the library's header
-    fixes them: chunk length = ceil(ceil(kv_len / S) / align) * align."""
+    fixes them: the edge between split s - 1 and split s is s * kv_len / S
+    rounded to the nearest multiple of align (ties up), at most kv_len; the
+    first split starts at 0 and the last ends at kv_len."""
     kv = kv_len.astype(np.int64)
-    chunk = ((kv + splits - 1) // splits + align - 1) // align * align
+    edges = [np.zeros_like(kv)]
+    for s in range(1, splits):
+        e = (2 * s * kv + splits * align) // (2 * splits * align) * align
+        edges.append(np.minimum(e, kv))
+    edges.append(kv)
     out = np.zeros((kv.shape[0], splits, 2), np.int32)
     for s in range(splits):
-        lo = np.minimum(s * chunk, kv)
-        hi = np.minimum((s + 1) * chunk, kv)
-        out[:, s, 0] = lo
-        out[:, s, 1] = hi
+        out[:, s, 0] = edges[s]
+        out[:, s, 1] = edges[s + 1]
     return out

@@ -30,6 +30,22 @@ def test_split_share_covers_every_split_once(S, world):
     assert max(counts) - min(counts) <= 1
 
 
+@pytest.mark.parametrize("S", [1, 2, 3, 5, 16, 64])
+def test_split_bounds_partition(S):
+    from speculative_decoding_tree_va_b200 import synth
+    kv = np.array([1, 33, 255, 256, 257, 2081, 4096, 8225, 65 * 64 * 20, 131071], np.int32)
+    b = synth.split_bounds(kv, S)
+    assert b.shape == (kv.size, S, 2)
+    for r in range(kv.size):
+        lo, hi = b[r, :, 0].astype(np.int64), b[r, :, 1].astype(np.int64)
+        assert lo[0] == 0 and hi[-1] == kv[r]
+        assert np.all(hi[:-1] == lo[1:]) and np.all(hi >= lo)   # contiguous, ordered
+        assert np.all((lo % 256 == 0) | (lo == kv[r]))            # every edge but kv_len aligned
+        exact = np.arange(S) * kv[r] / S                          # nearest multiple of 256
+        assert np.all(np.abs(lo[1:] - exact[1:]) <= 128)
+        assert np.all(np.abs((hi - lo) - kv[r] / S) < 256)
+
+
 def test_split_share_rejects_bad_arguments():
     for bad in ((0, 2, 0), (4, 0, 0), (4, 2, 2), (4, 2, -1)):
         with pytest.raises(ValueError):
