@@ -315,9 +315,11 @@ int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, in
 int va_verify_attn_noalloc(const va_attn_args* args, va_stream_t stream);
 
 /*
- * Diagnostic: number of bounded barrier waits inside the tensor-core kernel
- * that expired on the current device since the library was loaded (each
- * expiry also flags its request with VA_ERR_CUDA).  Synchronises the
+ * Diagnostic: number of bounded barrier waits inside the attention kernels
+ * (the tensor-core kernel's pipeline barriers, the CUDA-core kernel's
+ * bulk-copy staging of an fp32 cache) that expired on the current device
+ * since the library was loaded (each expiry also flags its request with
+ * VA_ERR_CUDA).  Synchronises the
  * device; returns 0xFFFFFFFF if the counter cannot be read.
  */
 unsigned int va_device_timeouts(void);

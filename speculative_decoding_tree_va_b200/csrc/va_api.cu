@@ -270,4 +270,10 @@ int va_merge(const float* o_part, const float* lse_part, int S, int B, int T, in
   return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
 }
 
+unsigned int va_device_timeouts(void) {
+  const unsigned int a = va::tc_timeouts(), b = va::simt_timeouts();
+  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return 0xFFFFFFFFu;
+  return a + b;
+}
+
 }  // extern "C"

@@ -9,8 +9,10 @@
 //
 // Layout: one CTA = 32 consecutive rows (row = t*H + h) of one request and one
 // key split, 8 warps; key tiles of 32 keys (all 576 q.k dims, fp32 in shared
-// memory, double-buffered; cp.async for fp32 inputs; the staged Q shares the
-// second key buffer, which is free until the second tile).  Per tile:
+// memory, double-buffered; the staged Q shares the second key buffer, which
+// is free until the second tile).  An fp32 cache is staged by bulk copies,
+// one c_kv row and one k_pe row per lane of warp 0, completed on an mbarrier
+// (bounded wait), so the staging costs the other warps nothing.  Per tile:
 //  * S = Q.K^T (32 x 16): warp w takes dims [72w, 72w + 72) of every row and
 //    key; lane (i, j) keeps the Q of rows i + 8a (a = 0..3) and dims
 //    [72w + 18j, +18) in registers for the whole key range and reads only K
@@ -29,9 +31,13 @@
 // inner loops are those of the other types.
 #include <cuda_fp8.h>
 
+#include "va_bulk.cuh"
 #include "va_common.cuh"
 
 namespace va {
+
+__device__ unsigned int g_simt_timeouts = 0;  // count of staging waits that expired
+
 namespace {
 
 constexpr int kRows = 32;       // rows per CTA
@@ -51,6 +57,8 @@ constexpr size_t kSmemTotal = 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof
 static_assert(kDqk % (8 * kWarps) == 0, "dims split evenly into float2 steps per lane");
 static_assert(kRows <= kKeys, "the staged Q fits in a key buffer");
 static_assert(kKeys % 8 == 0 && kKeys / 8 <= 8, "8-key groups in Q.K^T; 8 softmax lanes per row");
+static_assert(kKeys == 32, "bulk staging: one key row per lane of one warp");
+static_assert((kStride * sizeof(float)) % 16 == 0, "bulk copies land on 16-byte boundaries");
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -205,6 +213,10 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   float* sM = sAlpha + kRows;               // [row] final running max (log2 domain)
   float* sL = sM + kRows;                   // [row] final sum
   __shared__ int bad_page;
+  __shared__ int aborted;                   // a staging wait expired
+  __shared__ __align__(8) uint64_t kv_full; // bulk-staged tile t completes phase t
+  // an fp32 cache is staged by bulk copies; other types are widened on the way
+  constexpr bool kBulk = sizeof(Tkv) == 4;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -219,7 +231,14 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   int lo = 0, hi = 0;
   if (req_ok) split_range(kv_len, S, split0 + split, &lo, &hi);
   const int P = kv_len - T;
-  if (tid == 0) bad_page = 0;
+  if (tid == 0) {
+    bad_page = 0;
+    aborted = 0;
+    if (kBulk) {
+      bulk::mbar_init(&kv_full, 1);
+      bulk::fence_mbar_init();
+    }
+  }
   __syncthreads();
 
   // q rows -> shared (fp32).  Rows past R are zero.
@@ -270,20 +289,52 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     for (int c = 0; c < 4; ++c) acc[r][c] = make_float2(0.f, 0.f);
 
   const int ntiles = (hi > lo) ? (hi - lo + kKeys - 1) / kKeys : 0;
-  auto phys_of = [&](int j0) -> int {
-    const int pg = page_table[(size_t)b * max_pages + j0 / kPage];
+  // Page-table entries are read one tile ahead of their use, so the global
+  // load's latency does not sit between a tile's barrier and its staging.
+  auto page_of = [&](int j0) -> int { return page_table[(size_t)b * max_pages + j0 / kPage]; };
+  auto checked = [&](int pg) -> int {
     if (pg < 0 || pg >= num_pages) { bad_page = 1; return -1; }
     return pg;
   };
-  // fp32 keys go to shared memory by cp.async; other types through registers
-  constexpr bool kAsync = sizeof(Tkv) == 4;
+  auto phys_of = [&](int j0) -> int { return checked(page_of(j0)); };
+  int pg_ahead = ntiles > 1 ? page_of(lo + kKeys) : 0;  // entry of the tile being staged next
+  // Bulk staging of keys [j0, j0 + 32) (one page) into dst, called by every
+  // thread alike.  All 32 rows are copied: rows at or past `hi` lie in the
+  // same page, hold finite values, and get probability exactly 0.  A bad
+  // page instead zeroes the tile with plain stores and completes the phase
+  // without copies.
+  auto stage_bulk = [&](float* dst, int phys, int j0) {
+    if constexpr (kBulk) {
+      if (phys >= 0) {
+        if (warp == 0) {
+          bulk::fence_proxy_async();
+          if (lane == 0)
+            bulk::mbar_arrive_expect_tx(&kv_full, kKeys * (kDc + kDr) * (uint32_t)sizeof(float));
+          __syncwarp();
+          const size_t krow = (size_t)phys * kPage + (j0 & (kPage - 1)) + lane;
+          bulk::copy_g2s(dst + lane * kStride, c_kv + krow * kDc, kDc * sizeof(float), &kv_full);
+          bulk::copy_g2s(dst + lane * kStride + kDc, k_pe + krow * kDr, kDr * sizeof(float),
+                         &kv_full);
+        }
+      } else {
+        for (int c = tid; c < kKeys * kStride / 4; c += kThreads)
+          reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        bulk::fence_proxy_async();
+        if (tid == 0) bulk::mbar_arrive_expect_tx(&kv_full, 0);
+      }
+    }
+  };
   RegStage<Tkv> reg;
-  if (ntiles > 0) stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
-  cp_async_commit();
+  if (ntiles > 0) {
+    if constexpr (kBulk) stage_bulk(sK0, phys_of(lo), lo);
+    else stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
+  }
   // this lane's Q: rows qi + 8 a, dims [72 warp + 18 qj, +18), kept in
   // registers for every key tile
   float2 qr[4][kSub / 2];  // (even dim, odd dim) pairs
+  cp_async_commit();
   cp_async_wait_all();
+  if (kBulk) bulk::fence_proxy_async();  // the staged Q's buffer later takes bulk copies
   __syncthreads();
   {
     const float* qb = sQ + qi * kStride + warp * kDSlice + kSub * qj;
@@ -297,17 +348,29 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   for (int it = 0; it < ntiles; ++it) {
     float* sK = (it & 1) ? sK1 : sK0;
     float* sKn = (it & 1) ? sK0 : sK1;
-    cp_async_wait_all();
-    __syncthreads();  // tile it staged; the previous tile's P.V (and, at the
-                      // first tile, every read of the staged Q) is done
+    // tile it staged; the previous tile's P.V (and, at the first tile, every
+    // read of the staged Q) is done, so the other buffer is free
+    if constexpr (kBulk) {
+      const bool ok = bulk::mbar_wait(&kv_full, it & 1);
+      if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+          aborted = 1;
+          atomicAdd(&g_simt_timeouts, 1u);
+        }
+        bulk::settle();  // copies already issued land before the CTA moves on
+        break;
+      }
+    } else {
+      __syncthreads();
+    }
     const bool more = it + 1 < ntiles;
     const int jn = lo + (it + 1) * kKeys;
-    const int physn = more ? phys_of(jn) : -1;
+    const int physn = more ? checked(pg_ahead) : -1;
+    if (it + 2 < ntiles) pg_ahead = page_of(jn + kKeys);
     if (more) {
-      if (kAsync) stage_keys<Tkv>(sKn, c_kv, k_pe, physn, jn, hi, tid);
+      if constexpr (kBulk) stage_bulk(sKn, physn, jn);
       else reg.load(c_kv, k_pe, physn, jn, hi, tid, 0);
     }
-    cp_async_commit();
 
     // ---- partial scores of this warp's dim slice: the lane's Q rows stay in
     // registers (qr), only K comes from shared memory; the warp's four dim
@@ -365,7 +428,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     }
     // the other buffer is free (see the top of the loop): the first half of
     // the next tile goes in, the second half's loads overlap P.V
-    if (!kAsync && more) {
+    if (!kBulk && more) {
       reg.store(sKn, tid, 0);
       reg.load(c_kv, k_pe, physn, jn, hi, tid, 1);
     }
@@ -448,7 +511,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         }
       }
     }
-    if (!kAsync && more) reg.store(sKn, tid, 1);
+    if (!kBulk && more) reg.store(sKn, tid, 1);
   }
   cp_async_wait_all();
   if (sk == 0) {
@@ -456,7 +519,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     sL[sr] = l;
   }
   __syncthreads();
-  if (tid == 0 && req_status && (!req_ok || bad_page)) req_status[b] = VA_ERR_INVALID_ARG;
+  if (tid == 0 && req_status && (!req_ok || bad_page || aborted))
+    req_status[b] = aborted ? VA_ERR_CUDA : VA_ERR_INVALID_ARG;
 
   // epilogue: lane writes rows 8 pi + r, columns col0 .. +3 and col0 + 32 .. +3
   const size_t rows_total = (size_t)B * R;
@@ -466,8 +530,14 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     const int row = row0 + rr;
     if (row >= R) continue;
     const float lr = sL[rr];
-    const bool empty = !(lr > 0.f) || !req_ok || bad_page;
+    const bool empty = !(lr > 0.f) || !req_ok || bad_page || aborted;
+    // an expired wait leaves the accumulators undefined: multiply by 0 only
+    // what is known to be finite
     const float inv = empty ? 0.f : out_scale / lr;
+    if (aborted) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = make_float2(0.f, 0.f);
+    }
     const float lse = empty ? -INFINITY : (sM[rr] + log2f(lr)) * kLn2;
     const size_t g = (size_t)b * R + row;
     if (!o_part) {
@@ -510,6 +580,12 @@ cudaError_t launch_typed(const va_attn_args& a, SplitRange sp, float* o_part, fl
 }
 
 }  // namespace
+
+unsigned int simt_timeouts() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_simt_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  return v;
+}
 
 cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange S, float* o_part,
                              float* lse_part, cudaStream_t st) {

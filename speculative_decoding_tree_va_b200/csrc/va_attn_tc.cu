@@ -836,10 +836,10 @@ cudaError_t launch_attn_tc(const va_attn_args& a, SplitRange sp, const int32_t* 
   return cudaGetLastError();
 }
 
-}  // namespace va
-
-extern "C" unsigned int va_device_timeouts(void) {
+unsigned int tc_timeouts() {
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, va::g_tc_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  if (cudaMemcpyFromSymbol(&v, g_tc_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
   return v;
 }
+
+}  // namespace va

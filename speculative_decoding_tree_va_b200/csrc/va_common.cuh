@@ -113,6 +113,11 @@ cudaError_t launch_tree_accept(const int32_t* parents, const int32_t* tokens,
                                int32_t* accept_len, int32_t* next_token, cudaStream_t st);
 cudaError_t launch_tree_mask(const int32_t* parents, int B, int T, uint64_t* mask,
                              int32_t* status, cudaStream_t st);
+// Expired bounded waits of each attention kernel on the current device
+// (0xFFFFFFFF if the counter cannot be read).
+unsigned int tc_timeouts();
+unsigned int simt_timeouts();
+
 cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange sp, float* o_part,
                              float* lse_part, cudaStream_t st);
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
