@@ -10,12 +10,17 @@
 // Layout: one CTA = 32 consecutive rows (row = t*H + h) of one request and one
 // key split, 8 warps; key tiles of 32 keys (all 576 q.k dims, fp32 in shared
 // memory, double-buffered; the staged Q shares the second key buffer, which
-// is free until the second tile).  An fp32 cache is staged by bulk copies,
-// one c_kv row and one k_pe row per lane of warp 0, completed on an mbarrier
-// (bounded wait), so the staging costs the other warps nothing.  Per tile:
-//  * S = Q.K^T (32 x 16): warp w takes dims [72w, 72w + 72) of every row and
-//    key; lane (i, j) keeps the Q of rows i + 8a (a = 0..3) and dims
-//    [72w + 18j, +18) in registers for the whole key range and reads only K
+// is free until the second tile).  A staged tile is its 32 c_kv rows
+// ([32][512], dense) followed by its 32 k_pe rows ([32][64]): for an fp32
+// cache both parts are contiguous in the page, so warp 0 stages a tile with
+// nine bulk copies completed on an mbarrier (bounded wait), and the staging
+// costs the other warps nothing.  Per tile:
+//  * S = Q.K^T (32 x 32): warp w takes 72 of the 576 dims of every row and
+//    key: c_kv columns [64w, 64w + 64) and k_pe columns [8w, 8w + 8).  Lane
+//    (i, j) keeps the Q of rows i + 8a (a = 0..3) on its 18 of them in
+//    registers for the whole key range -- the column pairs 64w + 8m + 2j
+//    (m = 0..7) and k_pe pair 8w + 2j, so the four j lanes read adjacent
+//    pairs of a key row, conflict-free without padding -- and reads only K
 //    from shared memory (one 8-byte load feeds 8 FFMAs across its 4 rows);
 //    the four dim sub-slices of a warp are summed with shuffles, the 8
 //    warps' partial tiles through shared memory.
@@ -24,7 +29,8 @@
 //  * O += P.V (32 x 512): warp w owns columns [64w, 64w + 64), each lane an
 //    8-row x 8-column register tile, so two 16-byte loads of P and two of V
 //    feed 64 FFMAs.
-// Row strides of 580 floats keep the strided 16-byte reads conflict-free.
+// All lanes of a warp read the same key row in both products, so the dense
+// rows cause no bank conflicts there.
 //
 // FP8 cache: codes are widened to fp32 while they are staged; the cache scale
 // is folded into the score scale and into the output normalisation, so the
@@ -44,13 +50,12 @@ constexpr int kRows = 32;       // rows per CTA
 constexpr int kKeys = 32;       // keys per tile
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStride = kDqk + 4;          // floats per staged Q / K row
-constexpr int kDSlice = kDqk / kWarps;     // q.k dims per warp: 72
-constexpr int kSub = kDSlice / 4;          // dims per lane (four sub-slices per warp): 18
+constexpr int kSub = kDqk / kWarps / 4;   // dims per lane (four sub-slices per warp): 18
 constexpr int kSpStride = 36;              // partial-score tile [key][row], padded
 constexpr int kPStride = kRows + 4;        // probabilities [key][row], padded
 constexpr float kRescaleLog2 = 8.0f;       // lazy max: rescale only past 2^8
-constexpr size_t kSmemK = (size_t)kKeys * kStride * sizeof(float);
+constexpr int kTileFloats = kKeys * kDqk;  // one staged tile: [32][512] c_kv, then [32][64] k_pe
+constexpr size_t kSmemK = (size_t)kTileFloats * sizeof(float);
 constexpr size_t kSmemSp = (size_t)kWarps * kKeys * kSpStride * sizeof(float);
 constexpr size_t kSmemP = (size_t)kKeys * kPStride * sizeof(float);
 constexpr size_t kSmemTotal = 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof(float);
@@ -58,7 +63,13 @@ static_assert(kDqk % (8 * kWarps) == 0, "dims split evenly into float2 steps per
 static_assert(kRows <= kKeys, "the staged Q fits in a key buffer");
 static_assert(kKeys % 8 == 0 && kKeys / 8 <= 8, "8-key groups in Q.K^T; 8 softmax lanes per row");
 static_assert(kKeys == 32, "bulk staging: one key row per lane of one warp");
-static_assert((kStride * sizeof(float)) % 16 == 0, "bulk copies land on 16-byte boundaries");
+static_assert(kRows == kKeys, "the staged Q uses the tile layout");
+static_assert(kDc == 64 * kWarps && kDr == 8 * kWarps && kSub == 18,
+              "per warp: 64 c_kv columns and 8 k_pe columns, 8 + 1 pairs per lane");
+
+// Row `key` of the c_kv part / the k_pe part of a staged tile.
+__device__ __forceinline__ float* c_row(float* t, int key) { return t + key * kDc; }
+__device__ __forceinline__ float* r_row(float* t, int key) { return t + kKeys * kDc + key * kDr; }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -128,7 +139,7 @@ __device__ void stage_keys(float* sK, const Tin* __restrict__ c_kv, const Tin* _
   for (int c = tid; c < kKeys * kChunks; c += kThreads) {
     const int key = c / kChunks;
     const int part = c - key * kChunks;
-    float* dst = sK + key * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+    float* dst = part < kChunksC ? c_row(sK, key) + part * V : r_row(sK, key) + (part - kChunksC) * V;
     const int j = j0 + key;
     if (j < hi && phys >= 0) {
       const size_t krow = (size_t)phys * kPage + (j & (kPage - 1));
@@ -182,7 +193,8 @@ struct RegStage {
       const int c = h * (kTotal / 2) + tid + i * kThreads;
       if (c < (h + 1) * (kTotal / 2)) {
         const int key = c / kChunks, part = c - key * kChunks;
-        float* dst = sK + key * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+        float* dst =
+            part < kChunksC ? c_row(sK, key) + part * V : r_row(sK, key) + (part - kChunksC) * V;
         load_row_chunk(dst, reinterpret_cast<const Tin*>(&buf[i]));
       }
     }
@@ -205,9 +217,9 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
   float* sK0 = smem;
-  float* sK1 = sK0 + kKeys * kStride;       // also the staged Q until tile 1 is staged
+  float* sK1 = sK0 + kTileFloats;           // also the staged Q until tile 1 is staged
   float* sQ = sK1;
-  float* sSp = sK1 + kKeys * kStride;       // [warp][key][row] partial scores
+  float* sSp = sK1 + kTileFloats;           // [warp][key][row] partial scores
   float* sP = sSp + kWarps * kKeys * kSpStride;  // [key][row] probabilities
   float* sAlpha = sP + kKeys * kPStride;    // [row] rescale factor of this tile
   float* sM = sAlpha + kRows;               // [row] final running max (log2 domain)
@@ -247,7 +259,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     constexpr int kChunksC = kDc / V, kChunks = kChunksC + kDr / V;
     for (int c = tid; c < kRows * kChunks; c += kThreads) {
       const int r = c / kChunks, part = c - r * kChunks;
-      float* dst = sQ + r * kStride + (part < kChunksC ? part * V : kDc + (part - kChunksC) * V);
+      float* dst = part < kChunksC ? c_row(sQ, r) + part * V : r_row(sQ, r) + (part - kChunksC) * V;
       const int row = row0 + r;
       if (row < R) {
         const size_t g = (size_t)b * R + row;
@@ -299,25 +311,30 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   auto phys_of = [&](int j0) -> int { return checked(page_of(j0)); };
   int pg_ahead = ntiles > 1 ? page_of(lo + kKeys) : 0;  // entry of the tile being staged next
   // Bulk staging of keys [j0, j0 + 32) (one page) into dst, called by every
-  // thread alike.  All 32 rows are copied: rows at or past `hi` lie in the
-  // same page, hold finite values, and get probability exactly 0.  A bad
-  // page instead zeroes the tile with plain stores and completes the phase
-  // without copies.
+  // thread alike: lanes 0-7 of warp 0 copy 4 c_kv rows each (8 KB), lane 8
+  // the 32 k_pe rows (8 KB).  All 32 rows are copied: rows at or past `hi`
+  // lie in the same page, hold finite values, and get probability exactly
+  // 0.  A bad page instead zeroes the tile with plain stores and completes
+  // the phase without copies.
   auto stage_bulk = [&](float* dst, int phys, int j0) {
     if constexpr (kBulk) {
       if (phys >= 0) {
         if (warp == 0) {
           bulk::fence_proxy_async();
           if (lane == 0)
-            bulk::mbar_arrive_expect_tx(&kv_full, kKeys * (kDc + kDr) * (uint32_t)sizeof(float));
+            bulk::mbar_arrive_expect_tx(&kv_full, kTileFloats * (uint32_t)sizeof(float));
           __syncwarp();
-          const size_t krow = (size_t)phys * kPage + (j0 & (kPage - 1)) + lane;
-          bulk::copy_g2s(dst + lane * kStride, c_kv + krow * kDc, kDc * sizeof(float), &kv_full);
-          bulk::copy_g2s(dst + lane * kStride + kDc, k_pe + krow * kDr, kDr * sizeof(float),
-                         &kv_full);
+          const size_t krow = (size_t)phys * kPage + (j0 & (kPage - 1));
+          constexpr int kRowsPerCopy = kKeys / 8;
+          if (lane < 8)
+            bulk::copy_g2s(c_row(dst, kRowsPerCopy * lane),
+                           c_kv + (krow + kRowsPerCopy * lane) * kDc,
+                           kRowsPerCopy * kDc * sizeof(float), &kv_full);
+          else if (lane == 8)
+            bulk::copy_g2s(r_row(dst, 0), k_pe + krow * kDr, kKeys * kDr * sizeof(float), &kv_full);
         }
       } else {
-        for (int c = tid; c < kKeys * kStride / 4; c += kThreads)
+        for (int c = tid; c < kTileFloats / 4; c += kThreads)
           reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         bulk::fence_proxy_async();
         if (tid == 0) bulk::mbar_arrive_expect_tx(&kv_full, 0);
@@ -329,20 +346,22 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     if constexpr (kBulk) stage_bulk(sK0, phys_of(lo), lo);
     else stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
   }
-  // this lane's Q: rows qi + 8 a, dims [72 warp + 18 qj, +18), kept in
-  // registers for every key tile
-  float2 qr[4][kSub / 2];  // (even dim, odd dim) pairs
+  // this lane's Q: rows qi + 8 a, c_kv column pairs 64 warp + 8 m + 2 qj
+  // (m = 0..7) and k_pe pair 8 warp + 2 qj, kept in registers for every key
+  // tile
+  float2 qr[4][kSub / 2];  // (even dim, odd dim) pairs; [8] is the k_pe pair
   cp_async_commit();
   cp_async_wait_all();
   if (kBulk) bulk::fence_proxy_async();  // the staged Q's buffer later takes bulk copies
   __syncthreads();
   {
-    const float* qb = sQ + qi * kStride + warp * kDSlice + kSub * qj;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 4; ++a) {
+      const float* qc = c_row(sQ, qi + 8 * a) + 64 * warp + 2 * qj;
 #pragma unroll
-      for (int m2 = 0; m2 < kSub / 2; ++m2)
-        qr[a][m2] = *reinterpret_cast<const float2*>(qb + a * 8 * kStride + 2 * m2);
+      for (int m = 0; m < 8; ++m) qr[a][m] = *reinterpret_cast<const float2*>(qc + 8 * m);
+      qr[a][8] = *reinterpret_cast<const float2*>(r_row(sQ, qi + 8 * a) + 8 * warp + 2 * qj);
+    }
   }
 
   for (int it = 0; it < ntiles; ++it) {
@@ -386,13 +405,14 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int c = 0; c < 8; ++c) acc2[a][c] = make_float2(0.f, 0.f);
-        const float* kb = sK + (8 * half) * kStride + warp * kDSlice + kSub * qj;
+        const float* kc = c_row(sK, 8 * half) + 64 * warp + 2 * qj;
+        const float* kr = r_row(sK, 8 * half) + 8 * warp + 2 * qj;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float2 kv[kSub / 2];
 #pragma unroll
-          for (int m2 = 0; m2 < kSub / 2; ++m2)
-            kv[m2] = *reinterpret_cast<const float2*>(kb + c * kStride + 2 * m2);
+          for (int m = 0; m < 8; ++m) kv[m] = *reinterpret_cast<const float2*>(kc + c * kDc + 8 * m);
+          kv[8] = *reinterpret_cast<const float2*>(kr + c * kDr);
 #pragma unroll
           for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -498,8 +518,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
       for (int k = 0; k < kKeys; ++k) {
         const float4 p0 = *reinterpret_cast<const float4*>(sP + k * kPStride + 8 * pi);
         const float4 p1 = *reinterpret_cast<const float4*>(sP + k * kPStride + 8 * pi + 4);
-        const float4 v0 = *reinterpret_cast<const float4*>(sK + k * kStride + col0);
-        const float4 v1 = *reinterpret_cast<const float4*>(sK + k * kStride + col0 + 32);
+        const float4 v0 = *reinterpret_cast<const float4*>(c_row(sK, k) + col0);
+        const float4 v1 = *reinterpret_cast<const float4*>(c_row(sK, k) + col0 + 32);
         const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
         const float2 vv[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w),
                               make_float2(v1.x, v1.y), make_float2(v1.z, v1.w)};
