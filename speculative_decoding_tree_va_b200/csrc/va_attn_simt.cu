@@ -18,12 +18,15 @@
 //  * S = Q.K^T (32 x 32): warp w takes 72 of the 576 dims of every row and
 //    key: c_kv columns [64w, 64w + 64) and k_pe columns [8w, 8w + 8).  Lane
 //    (i, j) keeps the Q of rows i + 8a (a = 0..3) on its 18 of them in
-//    registers for the whole key range -- the column pairs 64w + 8m + 2j
-//    (m = 0..7) and k_pe pair 8w + 2j, so the four j lanes read adjacent
-//    pairs of a key row, conflict-free without padding -- and reads only K
-//    from shared memory (one 8-byte load feeds 8 FFMAs across its 4 rows);
-//    the four dim sub-slices of a warp are summed with shuffles, the 8
-//    warps' partial tiles through shared memory.
+//    registers for the whole key range -- the column quads 64w + 16m + 4j
+//    (m = 0..3) and k_pe pair 8w + 2j, so the four j lanes read adjacent
+//    16-byte chunks of a key row, conflict-free without padding -- and
+//    reads only K from shared memory (one 16-byte load feeds 16 FFMAs
+//    across its 4 rows).  The four dim sub-slices of a warp are summed by a
+//    two-step shuffle butterfly; each lane visits its 8 keys of a group in
+//    the order c ^ (4 j0 + 2 j1) (j = j0 + 2 j1), which makes the entries it
+//    keeps and gives the same at every lane, so the butterfly needs no
+//    selects.  The 8 warps' partial tiles are summed through shared memory.
 //  * softmax: 8 lanes per row, 4 keys each; the running max moves (and O is
 //    rescaled) only when a tile raises it by more than 2^8.
 //  * O += P.V (32 x 512): warp w owns columns [64w, 64w + 64), each lane an
@@ -346,8 +349,8 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     if constexpr (kBulk) stage_bulk(sK0, phys_of(lo), lo);
     else stage_keys<Tkv>(sK0, c_kv, k_pe, phys_of(lo), lo, hi, tid);
   }
-  // this lane's Q: rows qi + 8 a, c_kv column pairs 64 warp + 8 m + 2 qj
-  // (m = 0..7) and k_pe pair 8 warp + 2 qj, kept in registers for every key
+  // this lane's Q: rows qi + 8 a, c_kv column quads 64 warp + 16 m + 4 qj
+  // (m = 0..3) and k_pe pair 8 warp + 2 qj, kept in registers for every key
   // tile
   float2 qr[4][kSub / 2];  // (even dim, odd dim) pairs; [8] is the k_pe pair
   cp_async_commit();
@@ -357,9 +360,13 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
   {
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-      const float* qc = c_row(sQ, qi + 8 * a) + 64 * warp + 2 * qj;
+      const float* qc = c_row(sQ, qi + 8 * a) + 64 * warp + 4 * qj;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) qr[a][m] = *reinterpret_cast<const float2*>(qc + 8 * m);
+      for (int m = 0; m < 4; ++m) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qc + 16 * m);
+        qr[a][2 * m] = make_float2(q4.x, q4.y);
+        qr[a][2 * m + 1] = make_float2(q4.z, q4.w);
+      }
       qr[a][8] = *reinterpret_cast<const float2*>(r_row(sQ, qi + 8 * a) + 8 * warp + 2 * qj);
     }
   }
@@ -396,6 +403,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
     // sub-slices are summed with shuffles before the cross-warp reduction
     {
       const bool b0 = (qj & 1) != 0, b1 = (qj >> 1) != 0;
+      const int kmask = 4 * b0 + 2 * b1;  // this lane visits key c of a group as c ^ kmask
       float* sp = sSp + warp * kKeys * kSpStride;
 #pragma unroll
       for (int half = 0; half < kKeys / 8; ++half) {
@@ -405,43 +413,54 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int c = 0; c < 8; ++c) acc2[a][c] = make_float2(0.f, 0.f);
-        const float* kc = c_row(sK, 8 * half) + 64 * warp + 2 * qj;
-        const float* kr = r_row(sK, 8 * half) + 8 * warp + 2 * qj;
+        // rows of the key pairs (c & 6) ^ kmask of this group; c & 1 is a
+        // compile-time offset from them
+        const float* kcb[4];
+        const float* krb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          kcb[i] = c_row(sK, 8 * half + ((2 * i) ^ kmask)) + 64 * warp + 4 * qj;
+          krb[i] = r_row(sK, 8 * half + ((2 * i) ^ kmask)) + 8 * warp + 2 * qj;
+        }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
+          const float* kcc = kcb[c >> 1] + (c & 1) * kDc;
           float2 kv[kSub / 2];
 #pragma unroll
-          for (int m = 0; m < 8; ++m) kv[m] = *reinterpret_cast<const float2*>(kc + c * kDc + 8 * m);
-          kv[8] = *reinterpret_cast<const float2*>(kr + c * kDr);
+          for (int m = 0; m < 4; ++m) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kcc + 16 * m);
+            kv[2 * m] = make_float2(k4.x, k4.y);
+            kv[2 * m + 1] = make_float2(k4.z, k4.w);
+          }
+          kv[8] = *reinterpret_cast<const float2*>(krb[c >> 1] + (c & 1) * kDr);
 #pragma unroll
           for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int m2 = 0; m2 < kSub / 2; ++m2) acc2[a][c] = fma2(qr[a][m2], kv[m2], acc2[a][c]);
         }
+        // acc8[a][c]: row qi + 8a, key 8 half + (c ^ kmask), over this lane's dims
         float acc8[4][8];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int c = 0; c < 8; ++c) acc8[a][c] = acc2[a][c].x + acc2[a][c].y;
-        // lanes qi + 8 qj, qj = 0..3, hold the same rows and keys over four
-        // dim sub-slices: halve the keys per lane twice while summing pairs
+        // Lanes qi + 8 qj, qj = 0..3, hold the same rows over four dim
+        // sub-slices.  Step 1 (lane ^ 8 flips j0): entry c < 4 of both lanes
+        // is a key with bit 2 = j0 of this lane, entry 4 + c of the partner
+        // the same key; step 2 (lane ^ 16 flips j1) likewise on bit 1.
         float r1[4][4];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float mine = b0 ? acc8[a][4 + c] : acc8[a][c];
-            const float give = b0 ? acc8[a][c] : acc8[a][4 + c];
-            r1[a][c] = mine + __shfl_xor_sync(0xffffffffu, give, 8);
-          }
+          for (int c = 0; c < 4; ++c)
+            r1[a][c] = acc8[a][c] + __shfl_xor_sync(0xffffffffu, acc8[a][4 + c], 8);
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const float mine = b1 ? r1[a][2 + c] : r1[a][c];
-            const float give = b1 ? r1[a][c] : r1[a][2 + c];
-            const float v = mine + __shfl_xor_sync(0xffffffffu, give, 16);
-            // keys 8 half + 4 b0 + 2 b1 + c of row qi + 8 a, over the warp's dims
+            const float v = r1[a][c] + __shfl_xor_sync(0xffffffffu, r1[a][2 + c], 16);
+            // key 8 half + (c ^ kmask) = 8 half + 4 b0 + 2 b1 + c of row qi + 8 a,
+            // over the warp's dims
             sp[(8 * half + 4 * b0 + 2 * b1 + c) * kSpStride + qi + 8 * a] = v;
           }
       }
