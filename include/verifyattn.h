@@ -214,7 +214,8 @@ typedef struct va_attn_args {
  */
 size_t va_workspace_bytes(const va_attn_args* args);
 
-/* The split count va_verify_attn will use for these arguments (>= 1), or a
+/* The split count va_verify_attn will use for these arguments (>= 1; for
+ * the balanced CUDA-core plan below, the number of partials per row), or a
  * negative va_status on bad arguments. */
 int va_num_splits(const va_attn_args* args);
 
@@ -235,6 +236,16 @@ int va_num_splits(const va_attn_args* args);
  * + 256 S) / (512 S))), i.e. s * kv_len / S rounded to the nearest multiple
  * of 256, ties up (splits may be empty when kv_len < 128 S); the partials go
  * to the workspace and va_merge combines them on the same stream.
+ * Balanced plan: a call on the CUDA-core kernel with num_splits = 0 whose
+ * (request, 32-row tile) segments are fewer than the device's SMs instead
+ * cuts each segment's key range into 2 * max_pages 32-key tiles and divides
+ * the tiles of all segments, in order, into equal contiguous ranges, one CTA
+ * each (at least 4 tiles per CTA; none of this when that leaves no more CTAs
+ * than segments).  Every CTA writes one partial per segment it touches, a
+ * segment's unused slots are marked empty, and va_merge combines S = the
+ * largest number of CTAs sharing a segment (<= VA_MAX_SPLITS) partials.  The
+ * result is the same function of the inputs; only the fp32 rounding order
+ * differs.  va_verify_attn_partials never uses this plan.
  * bf16 runs on tensor cores with fp32 accumulation; fp32, and any call with
  * an FP8 cache (VA_FLAG_KV_FP8_E4M3), on CUDA cores.
  * Requirements: page_size == 64, H >= 1, 1 <= T <= 65, 0 <= B <= VA_MAX_BATCH

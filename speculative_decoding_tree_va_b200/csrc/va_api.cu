@@ -72,10 +72,13 @@ int check_args(const va_attn_args* a, bool needs_out = true) {
 // Split count: the caller's, or (num_splits == 0) the smallest power of two
 // that fills >= 90% of the last wave, keeping >= 1024 keys per split.  The
 // host does not see kv_len, so the planner uses the page-table capacity as
-// the key count.
+// the key count.  A CUDA-core call with fewer segments than SMs uses the
+// balanced plan instead (va_common.cuh), and its count is the plan's slots.
 int plan_splits(const va_attn_args* a) {
   if (a->num_splits > 0) return a->num_splits;
   if (a->B == 0) return 1;
+  const va::Balance bal = va::plan_balance(*a, sm_count());
+  if (bal.G) return bal.slots;
   const long long rows = (long long)a->T * a->H;
   long long units_per_split, slots;
   const int sms = sm_count();
@@ -106,7 +109,7 @@ namespace {
 // request order, when they apply): splits sp of the partition, partials to
 // o_part / lse_part (nullptr: a single split writing out / lse directly).
 int launch_attention(const va_attn_args& a, SplitRange sp, const WorkspaceLayout& w, char* base,
-                     float* o_part, float* lse_part, cudaStream_t st) {
+                     float* o_part, float* lse_part, cudaStream_t st, const Balance& bal) {
   cudaError_t e;
   const int32_t* order = nullptr;
   if (uses_tensor_cores(a)) {
@@ -134,7 +137,7 @@ int launch_attention(const va_attn_args& a, SplitRange sp, const WorkspaceLayout
   } else if (uses_tensor_cores(a)) {
     e = launch_attn_tc(a, sp, order, o_part, lse_part, st, 1.f);
   } else {
-    e = launch_attn_simt(a, sp, o_part, lse_part, st);
+    e = launch_attn_simt(a, sp, o_part, lse_part, st, bal);
   }
   if (e == cudaErrorNotSupported) return VA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return VA_ERR_CUDA;
@@ -148,7 +151,11 @@ int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
   char* base = static_cast<char*>(ws);
   float* o_part = S > 1 ? reinterpret_cast<float*>(base + w.o_part) : nullptr;
   float* lse_part = S > 1 ? reinterpret_cast<float*>(base + w.lse_part) : nullptr;
-  const int r = launch_attention(a, SplitRange{S, 0, S}, w, base, o_part, lse_part, st);
+  // the balanced plan is a function of the arguments and the device, so it is
+  // the one the split count S came from
+  const Balance bal = plan_balance(a, sm_count());
+  if (bal.G && bal.slots != S) return VA_ERR_INVALID_ARG;
+  const int r = launch_attention(a, SplitRange{S, 0, S}, w, base, o_part, lse_part, st, bal);
   if (r != VA_OK) return r;
   if (S > 1) {
     cudaError_t e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out,
@@ -161,7 +168,7 @@ int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
 int run_partials(const va_attn_args& a, SplitRange sp, void* ws, float* o_part, float* lse_part,
                  cudaStream_t st) {
   const WorkspaceLayout w = workspace_layout(a, sp.S, false);
-  return launch_attention(a, sp, w, static_cast<char*>(ws), o_part, lse_part, st);
+  return launch_attention(a, sp, w, static_cast<char*>(ws), o_part, lse_part, st, Balance{});
 }
 
 }  // namespace va

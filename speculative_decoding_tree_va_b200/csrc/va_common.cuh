@@ -104,6 +104,55 @@ struct SplitRange {
   int S, first, count;
 };
 
+// Balanced plan of the CUDA-core kernel for a full call (automatic split
+// count) whose (request, 32-row tile) segments are fewer than the SMs: each
+// segment's key range is cut into VT virtual 32-key tiles (VT = 2 max_pages,
+// the page table's capacity; tiles past kv_len are empty), the Q * VT tiles of
+// all segments in order are divided into G contiguous ranges of equal length,
+// one CTA each, and every CTA that covers part of a segment writes one
+// partial for it (slot = CTA - first CTA of the segment).  `slots` is the
+// largest number of CTAs that share a segment; the last CTA of a segment
+// marks its unused slots empty (lse -inf), and the merge combines `slots`
+// partials per row.  G = 0: not used (one CTA per segment and split).
+struct Balance {
+  int G = 0, VT = 0, NRT = 0, slots = 0;
+  long long U = 0;
+};
+// The CTA whose range holds virtual tile u: CTA c covers [c U / G, (c+1) U / G).
+__host__ __device__ __forceinline__ int balance_cta_of(long long u, long long U, int G) {
+  return (int)((u * G + G - 1) / U);
+}
+inline Balance plan_balance(const va_attn_args& a, int sms) {
+  Balance bal;
+  if (uses_tensor_cores(a) || a.num_splits != 0 || a.B < 1) return bal;
+  const int nrt = (a.T * a.H + 31) / 32;
+  const long long q = (long long)a.B * nrt;
+  if (q >= sms) return bal;  // one CTA per segment already fills the SMs
+  const int vt = 2 * a.max_pages;
+  const long long U = q * vt;
+  constexpr int kMinTilesPerCta = 4;
+  int G = sms;
+  if (U < (long long)G * kMinTilesPerCta) G = (int)(U / kMinTilesPerCta);
+  if (G <= q) return bal;  // no gain over one CTA per segment
+  for (; G > q; --G) {  // at most VA_MAX_SPLITS partials per row
+    int slots = 0;
+    for (long long s = 0; s < q; ++s) {
+      const int n = balance_cta_of((s + 1) * vt - 1, U, G) - balance_cta_of(s * vt, U, G) + 1;
+      slots = n > slots ? n : slots;
+    }
+    if (slots <= VA_MAX_SPLITS) {
+      if (slots < 2) return bal;
+      bal.G = G;
+      bal.VT = vt;
+      bal.NRT = nrt;
+      bal.slots = slots;
+      bal.U = U;
+      return bal;
+    }
+  }
+  return bal;
+}
+
 // Launchers implemented in the .cu files (internal C++ linkage).
 cudaError_t launch_build_tree(const double* lp, const int32_t* tok, int B, int L, int K,
                               int budget, int32_t* parents, int32_t* tokens, int32_t* depth,
@@ -119,7 +168,7 @@ unsigned int tc_timeouts();
 unsigned int simt_timeouts();
 
 cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange sp, float* o_part,
-                             float* lse_part, cudaStream_t st);
+                             float* lse_part, cudaStream_t st, const Balance& bal);
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
                          int out_dtype, void* out, float* lse, cudaStream_t st);
 cudaError_t launch_request_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t st);

@@ -121,6 +121,52 @@ def test_split_planning_and_workspace(lib):
     assert lib.va_num_splits(ctypes.byref(args(T=66))) == -va.VA_ERR_INVALID_ARG
 
 
+def _balanced_slots_brute_force(B, T, H, max_pages, sms=148):
+    """Partials per row of the balanced CUDA-core plan, by listing every CTA's
+    tile range: segments = B * ceil(T H / 32), 2 max_pages virtual tiles each,
+    G = min(sms, tiles / 4) CTAs (fewer while a segment would need more than
+    64 partials); None where the plan does not apply."""
+    q = B * (-(-T * H // 32))
+    if q >= sms:
+        return None
+    vt = 2 * max_pages
+    U = q * vt
+    G = min(sms, U // 4)
+    while G > q:
+        owners = [set() for _ in range(q)]
+        for c in range(G):
+            for u in range(c * U // G, (c + 1) * U // G):
+                owners[u // vt].add(c)
+        assert sum(len(o) for o in owners) >= q
+        slots = max(len(o) for o in owners)
+        if slots <= 64:
+            return slots if slots >= 2 else None
+        G -= 1
+    return None
+
+
+@pytest.mark.parametrize("B,T,H,max_pages", [
+    (1, 33, 64, 33),    # the fp32 page-test shape
+    (3, 21, 5, 15),     # partial row tiles
+    (1, 1, 1, 63),      # one 1-row segment
+    (2, 65, 2, 48),
+    (4, 9, 32, 2),      # too few tiles per CTA: the plain planner
+    (1, 65, 64, 2050),  # a long prefix with 131 segments
+])
+def test_balanced_cuda_core_plan(lib, B, T, H, max_pages):
+    """Without a device the planner takes 148 SMs, like a B200."""
+    want = _balanced_slots_brute_force(B, T, H, max_pages)
+    for kw in (dict(dtype=va.VA_F32), dict(flags=va.VA_FLAG_BF16_CUDA_CORES)):
+        got = lib.va_num_splits(ctypes.byref(args(B=B, T=T, H=H, max_pages=max_pages, **kw)))
+        if want is None:
+            assert got >= 1 and (got & (got - 1)) == 0  # the power-of-two planner
+        else:
+            assert got == want, (B, T, H, max_pages, kw)
+    # the tensor-core kernel never takes the balanced plan
+    tc = lib.va_num_splits(ctypes.byref(args(B=B, T=T, H=H, max_pages=max_pages)))
+    assert tc >= 1 and (tc & (tc - 1)) == 0  # the power-of-two planner
+
+
 def test_fp8_cache_split_planning_and_workspace(lib):
     """An FP8 cache keeps the query type's kernel (bf16: tensor cores, fp32: CUDA
     cores), so the auto split count is that kernel's; bf16 on the tensor cores

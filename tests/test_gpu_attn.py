@@ -147,6 +147,35 @@ def test_edge_cases(va, dtype, path, case):
     check_full(va, inp, path, what=f"{case}")
 
 
+# CUDA-core calls with fewer (request, 32-row tile) segments than SMs and an
+# automatic split count take the balanced plan: contiguous ranges of 32-key
+# tiles over one CTA per SM, a segment's partials in up to `slots` slots.
+BALANCED = [
+    dict(P=(5, 900), budget=20, topk=3, B=3, H=5),   # ragged lengths, partial row tiles
+    dict(P=4000, budget=0, H=1, B=1),                  # one 1-row segment over ~30 CTAs
+    dict(P=(1, 3000), budget=64, topk=2, H=2, B=2),   # T = 65, two mask words
+    dict(P=(300, 330), budget=8, H=32, B=4),          # kv_len below the page capacity
+]
+
+
+@pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "cc")])
+@pytest.mark.parametrize("case", BALANCED)
+def test_balanced_plan_matches_the_oracle(va, dtype, path, case):
+    import torch
+    inp = edge_inputs(dtype, **case)
+    if case.get("P") == (300, 330):
+        inp.kv_len[:] = np.minimum(inp.kv_len, inp.kv_len.min())  # empty tiles at every tail
+    d = to_device(inp, trees_for(inp)["parent"])
+    mask, _ = va.build_tree_mask(d["parents"])
+    out = torch.empty(*d["q_nope"].shape, dtype=d["q_nope"].dtype, device="cuda")
+    lse = torch.empty(*d["q_nope"].shape[:3], dtype=torch.float32, device="cuda")
+    flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
+    args = va.make_args(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], d["page_table"], d["kv_len"],
+                        mask, out, lse, scale=synth.SCALE, num_splits=0, flags=flags)
+    assert va.num_splits(args) > 1
+    check_full(va, inp, path, num_splits=0, what=f"balanced {case}")
+
+
 @pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
 @pytest.mark.parametrize("shape", ["chain", "star"])
 def test_chain_and_star_trees(va, dtype, path, shape):
