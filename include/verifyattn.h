@@ -180,6 +180,14 @@ typedef struct va_attn_args {
  * is in flight when the CTAs give up, so nothing lands after they exit. */
 #define VA_FLAG_TEST_STALL_MMA 2
 
+/* Test hook for the CUDA-core kernel's bounded staging wait (fp32 queries on
+ * an fp32 cache only; rejected with VA_ERR_INVALID_ARG elsewhere): the kernel
+ * arms each tile's staging barrier but issues no bulk copy, so the wait runs
+ * into its 1 s bound.  Each request then comes back with req_status
+ * VA_ERR_CUDA, zero output and lse -inf, va_device_timeouts() grows, and the
+ * context stays usable.  No copy is in flight when the CTAs give up. */
+#define VA_FLAG_TEST_STALL_COPIES 8
+
 /* Latent cache kept as FP8 E4M3 codes, one byte per element, with one scale
  * for the whole cache: c_kv is uint8 [num_pages, 64, 512], k_pe uint8
  * [num_pages, 64, 64], and code x stands for kv_scale * value(x) in every

@@ -22,6 +22,7 @@ VA_OK, VA_ERR_INVALID_ARG, VA_ERR_UNSUPPORTED, VA_ERR_CUDA, VA_ERR_INVALID_TREE 
 VA_F32, VA_BF16 = 0, 1
 VA_FLAG_BF16_CUDA_CORES = 1
 VA_FLAG_TEST_STALL_MMA = 2  # test hook: the tensor-core kernel's bounded waits expire
+VA_FLAG_TEST_STALL_COPIES = 8  # test hook: the CUDA-core kernel's staging waits expire
 VA_FLAG_KV_FP8_E4M3 = 4     # latent cache as FP8 E4M3 codes times kv_scale
 D_LATENT, D_ROPE, PAGE_SIZE, MAX_QLEN = 512, 64, 64, 65
 

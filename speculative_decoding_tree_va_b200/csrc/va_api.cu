@@ -44,8 +44,12 @@ int check_args(const va_attn_args* a, bool needs_out = true) {
   if (a->page_size != VA_PAGE_SIZE) return VA_ERR_UNSUPPORTED;
   if (a->B > VA_MAX_BATCH) return VA_ERR_UNSUPPORTED;  // the launches' request axis (grid y)
   if (a->num_splits < 0 || a->num_splits > VA_MAX_SPLITS) return VA_ERR_INVALID_ARG;
-  if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA | VA_FLAG_KV_FP8_E4M3))
+  if (a->flags & ~(VA_FLAG_BF16_CUDA_CORES | VA_FLAG_TEST_STALL_MMA | VA_FLAG_KV_FP8_E4M3 |
+                   VA_FLAG_TEST_STALL_COPIES))
     return VA_ERR_INVALID_ARG;
+  if ((a->flags & VA_FLAG_TEST_STALL_COPIES) &&
+      (a->dtype != VA_F32 || (a->flags & (VA_FLAG_KV_FP8_E4M3 | VA_FLAG_TEST_STALL_MMA))))
+    return VA_ERR_INVALID_ARG;  // only the bulk-staged fp32 cache has the hook
   if ((a->flags & VA_FLAG_TEST_STALL_MMA) &&
       (!va::uses_tensor_cores(*a) || (a->flags & VA_FLAG_KV_FP8_E4M3)))
     return VA_ERR_INVALID_ARG;  // only the tensor-core kernel on a bf16 cache has the hook

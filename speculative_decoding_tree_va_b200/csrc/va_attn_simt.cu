@@ -216,7 +216,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
                  const int32_t* __restrict__ page_table, int max_pages,
                  const int32_t* __restrict__ kv_len_arr, const uint64_t* __restrict__ tree_mask,
                  int H, int T, float scale_log2, float out_scale, int S, int split0,
-                 Balance bal, Tout* __restrict__ out,
+                 Balance bal, int stall_copies, Tout* __restrict__ out,
                  float* __restrict__ lse_out, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int32_t* __restrict__ req_status, int B) {
   extern __shared__ __align__(16) float smem[];
@@ -368,7 +368,9 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
             __syncwarp();
             const size_t krow = (size_t)phys * kPage + (j0 & (kPage - 1));
             constexpr int kRowsPerCopy = kKeys / 8;
-            if (lane < 8)
+            if (stall_copies) {
+              // test hook: the barrier expects the bytes, no copy brings them
+            } else if (lane < 8)
               bulk::copy_g2s(c_row(dst, kRowsPerCopy * lane),
                              c_kv + (krow + kRowsPerCopy * lane) * kDc,
                              kRowsPerCopy * kDc * sizeof(float), &kv_full);
@@ -664,7 +666,8 @@ cudaError_t launch_typed(const va_attn_args& a, SplitRange sp, float* o_part, fl
   kern<<<grid, kThreads, kSmemTotal, st>>>(
       (const Tq*)a.q_nope, (const Tq*)a.q_pe, (const Tkv*)a.c_kv, (const Tkv*)a.k_pe,
       a.num_pages, a.page_table, a.max_pages, a.kv_len, a.tree_mask, a.H, a.T, scale_log2,
-      kv_scale, sp.S, sp.first, bal, (Tout*)a.out, a.lse, o_part, lse_part, a.req_status, a.B);
+      kv_scale, sp.S, sp.first, bal, (a.flags & VA_FLAG_TEST_STALL_COPIES) ? 1 : 0, (Tout*)a.out,
+      a.lse, o_part, lse_part, a.req_status, a.B);
   return cudaGetLastError();
 }
 

@@ -60,7 +60,7 @@ def args(**kw):
     (dict(H=0), va.VA_ERR_INVALID_ARG), (dict(dtype=7), va.VA_ERR_INVALID_ARG),
     (dict(page_size=32), va.VA_ERR_UNSUPPORTED), (dict(num_splits=65), va.VA_ERR_INVALID_ARG),
     (dict(q_nope=None), va.VA_ERR_INVALID_ARG), (dict(c_kv=(1 << 20) + 8), va.VA_ERR_INVALID_ARG),
-    (dict(flags=8), va.VA_ERR_INVALID_ARG), (dict(num_pages=0), va.VA_ERR_INVALID_ARG),
+    (dict(flags=16), va.VA_ERR_INVALID_ARG), (dict(num_pages=0), va.VA_ERR_INVALID_ARG),
     (dict(num_splits=4), va.VA_ERR_INVALID_ARG),  # split without a workspace
     (dict(scale=float("nan")), va.VA_ERR_INVALID_ARG),
     (dict(B=65536), va.VA_ERR_UNSUPPORTED),     # beyond the launches' request axis
@@ -73,6 +73,13 @@ def args(**kw):
     (dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=float("nan")), va.VA_ERR_INVALID_ARG),
     (dict(flags=va.VA_FLAG_KV_FP8_E4M3, kv_scale=float("inf")), va.VA_ERR_INVALID_ARG),
     (dict(flags=va.VA_FLAG_KV_FP8_E4M3 | va.VA_FLAG_TEST_STALL_MMA, kv_scale=0.5),
+     va.VA_ERR_INVALID_ARG),
+    # the staging-wait hook exists only for fp32 queries on an fp32 cache
+    (dict(flags=va.VA_FLAG_TEST_STALL_COPIES), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_TEST_STALL_COPIES | va.VA_FLAG_BF16_CUDA_CORES), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_TEST_STALL_COPIES | va.VA_FLAG_KV_FP8_E4M3, kv_scale=0.5,
+          dtype=va.VA_F32), va.VA_ERR_INVALID_ARG),
+    (dict(flags=va.VA_FLAG_TEST_STALL_COPIES | va.VA_FLAG_TEST_STALL_MMA, dtype=va.VA_F32),
      va.VA_ERR_INVALID_ARG),
 ])
 def test_verify_attn_host_checks(lib, bad, status):
