@@ -329,7 +329,7 @@ attn_simt_kernel(const Tq* __restrict__ q_nope, const Tq* __restrict__ q_pe,
         live = mask_bit(mrow, t);
       }
     }
-    // Q.K^T role: rows qi + 8a (a = 0..3), dims [72 warp + 18 qj, +18), all keys.
+    // Q.K^T role: rows qi + 8a (a = 0..3), this warp's dims of sub-slice qj, all keys.
     const int qi = lane & 7, qj = lane >> 3;
     // P.V role: rows 8 pi .. 8 pi + 7; columns 64 warp + 4 pj + {0..3} and +32.
     const int pi = lane >> 3, pj = lane & 7;
