@@ -158,8 +158,10 @@ typedef struct va_attn_args {
   void* out;          /* [device] [B, T, H, 512] dtype, normalised latent out   */
   float* lse;         /* [device] [B, T, H] float, natural-log sum-exp          */
   int32_t* req_status;/* [device] [B] nullable: VA_ERR_INVALID_ARG when kv_len
-                         or a page index is out of range (rows written as 0 /
-                         -inf)                                                 */
+                         or a page index is out of range (all the request's
+                         rows written as 0 / -inf, with or without splits);
+                         entries of requests without a problem are not
+                         written                                               */
   int num_splits;     /* 0 = auto, 1 = single pass, 2..64 = split-KV + merge    */
   void* workspace;    /* [device] >= va_workspace_bytes(), 256-byte aligned     */
   size_t workspace_bytes;
@@ -214,7 +216,8 @@ typedef struct va_attn_args {
  *     order, int32 [B] (written by the call itself; the longest requests are
  *     scheduled first so the launch does not end on one long request);
  *   - for S > 1: o_part float [S, B, T, H, 512], then lse_part float
- *     [S, B, T, H] (the layout va_merge reads);
+ *     [S, B, T, H] (the layout va_merge reads), then int32 [B]: the splits'
+ *     per-request status, zeroed and filled by the call itself;
  *   - for bf16 queries on the tensor cores with an FP8 cache: the widened
  *     cache, bf16 [B * max_pages, 64, 512] and [B * max_pages, 64, 64], and
  *     its page table int32 [B, max_pages].

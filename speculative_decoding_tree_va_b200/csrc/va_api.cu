@@ -159,14 +159,21 @@ int run_verify(const va_attn_args& a, int S, void* ws, cudaStream_t st) {
   // the one the split count S came from
   const Balance bal = plan_balance(a, sm_count());
   if (bal.G && bal.slots != S) return VA_ERR_INVALID_ARG;
-  const int r = launch_attention(a, SplitRange{S, 0, S}, w, base, o_part, lse_part, st, bal);
+  if (S == 1) return launch_attention(a, SplitRange{1, 0, 1}, w, base, nullptr, nullptr, st, bal);
+  // Split: a request flagged by one split (a bad page, an expired wait) must
+  // come out empty although its other splits hold partials, so the splits
+  // report into the call's own status array and the merge empties flagged
+  // requests and passes their status on to the caller's array.
+  int32_t* status = reinterpret_cast<int32_t*>(base + w.status);
+  if (cudaMemsetAsync(status, 0, (size_t)a.B * sizeof(int32_t), st) != cudaSuccess)
+    return VA_ERR_CUDA;
+  va_attn_args as = a;
+  as.req_status = status;
+  const int r = launch_attention(as, SplitRange{S, 0, S}, w, base, o_part, lse_part, st, bal);
   if (r != VA_OK) return r;
-  if (S > 1) {
-    cudaError_t e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out,
-                                 a.lse, st);
-    if (e != cudaSuccess) return VA_ERR_CUDA;
-  }
-  return VA_OK;
+  cudaError_t e = launch_merge(o_part, lse_part, S, (long long)a.B * a.T * a.H, a.dtype, a.out,
+                               a.lse, st, status, a.T * a.H, a.req_status);
+  return e == cudaSuccess ? VA_OK : VA_ERR_CUDA;
 }
 
 int run_partials(const va_attn_args& a, SplitRange sp, void* ws, float* o_part, float* lse_part,

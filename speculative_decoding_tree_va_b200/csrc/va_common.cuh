@@ -59,19 +59,20 @@ inline bool widens_fp8_cache(const va_attn_args& a) {
 
 // Workspace layout of one call: on the tensor-core path, the requests'
 // longest-first order (int32 [B]); then the split-KV partials (S > 1 and not
-// a partials-only call, whose partials go to the caller's arrays); then the
+// a partials-only call, whose partials go to the caller's arrays) and the
+// call's own per-request status (int32 [B], same condition); then the
 // widened cache (widens_fp8_cache): bf16 [B * max_pages, 64, 512], bf16
 // [B * max_pages, 64, 64] and an int32 [B, max_pages] page table.  Every part
 // starts on a 256-byte boundary.  Offsets are in bytes; `total` is 0 when
 // nothing is needed.
 struct WorkspaceLayout {
-  size_t order, o_part, lse_part, w_ckv, w_kpe, w_table, total;
+  size_t order, o_part, lse_part, status, w_ckv, w_kpe, w_table, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S, bool partials_here = true) {
-  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0};
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0, 0};
   const size_t rows = (size_t)a.B * a.T * a.H;
   size_t off = 0;
   if (uses_tensor_cores(a)) {
@@ -83,6 +84,8 @@ inline WorkspaceLayout workspace_layout(const va_attn_args& a, int S, bool parti
     off += align256((size_t)S * rows * kDc * sizeof(float));
     w.lse_part = off;
     off += align256((size_t)S * rows * sizeof(float));
+    w.status = off;
+    off += align256((size_t)a.B * sizeof(int32_t));
   }
   if (widens_fp8_cache(a)) {
     const size_t pages = (size_t)a.B * a.max_pages;
@@ -169,8 +172,13 @@ unsigned int simt_timeouts();
 
 cudaError_t launch_attn_simt(const va_attn_args& a, SplitRange sp, float* o_part,
                              float* lse_part, cudaStream_t st, const Balance& bal);
+// req_bad (nullable): per-request status of the attention launches; every row
+// of a request with a non-zero status is written as 0 / -inf, and the status
+// is copied into req_status (nullable) at that request.
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
-                         int out_dtype, void* out, float* lse, cudaStream_t st);
+                         int out_dtype, void* out, float* lse, cudaStream_t st,
+                         const int32_t* req_bad = nullptr, int rows_per_req = 1,
+                         int32_t* req_status = nullptr);
 cudaError_t launch_request_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t st);
 cudaError_t launch_attn_tc(const va_attn_args& a, SplitRange sp, const int32_t* order,
                            float* o_part, float* lse_part, cudaStream_t st, float out_scale);

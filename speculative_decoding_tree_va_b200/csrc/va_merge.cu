@@ -32,10 +32,26 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4
 template <typename Tout>
 __global__ void __launch_bounds__(kWarps * 32)
 merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, int S,
-             long long rows, Tout* __restrict__ out, float* __restrict__ lse) {
+             long long rows, Tout* __restrict__ out, float* __restrict__ lse,
+             const int32_t* __restrict__ req_bad, int rows_per_req,
+             int32_t* __restrict__ req_status) {
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
+  if (req_bad) {  // a flagged request's rows come out empty, whatever its other splits hold
+    const long long b = row / rows_per_req;
+    const int32_t st = req_bad[b];
+    if (st != 0) {
+      Tout* orow = out + row * kDc + lane * 4;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) store4<Tout>(orow + g * 128, make_float4(0.f, 0.f, 0.f, 0.f));
+      if (lane == 0) {
+        lse[row] = -INFINITY;
+        if (req_status && row == b * rows_per_req) req_status[b] = st;
+      }
+      return;
+    }
+  }
   // S <= 64: lanes hold chunks lane and lane + 32.
   const float l0 = lane < S ? lse_part[(long long)lane * rows + row] : -INFINITY;
   const float l1 = lane + 32 < S ? lse_part[(long long)(lane + 32) * rows + row] : -INFINITY;
@@ -79,15 +95,16 @@ merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_par
 }  // namespace
 
 cudaError_t launch_merge(const float* o_part, const float* lse_part, int S, long long rows,
-                         int out_dtype, void* out, float* lse, cudaStream_t st) {
+                         int out_dtype, void* out, float* lse, cudaStream_t st,
+                         const int32_t* req_bad, int rows_per_req, int32_t* req_status) {
   if (rows == 0) return cudaSuccess;
   const long long blocks = (rows + kWarps - 1) / kWarps;
   if (out_dtype == VA_F32)
-    merge_kernel<float><<<(unsigned)blocks, kWarps * 32, 0, st>>>(o_part, lse_part, S, rows,
-                                                                  (float*)out, lse);
+    merge_kernel<float><<<(unsigned)blocks, kWarps * 32, 0, st>>>(
+        o_part, lse_part, S, rows, (float*)out, lse, req_bad, rows_per_req, req_status);
   else
     merge_kernel<__nv_bfloat16><<<(unsigned)blocks, kWarps * 32, 0, st>>>(
-        o_part, lse_part, S, rows, (__nv_bfloat16*)out, lse);
+        o_part, lse_part, S, rows, (__nv_bfloat16*)out, lse, req_bad, rows_per_req, req_status);
   return cudaGetLastError();
 }
 

@@ -107,12 +107,13 @@ def test_other_host_checks(lib):
 
 def test_split_planning_and_workspace(lib):
     # tensor cores: the request order (int32 [B]) first; explicit split count:
-    # partials [S,B,T,H,512] f32 + [S,B,T,H] f32; every part 256-byte aligned
+    # partials [S,B,T,H,512] f32 + [S,B,T,H] f32 + the splits' status int32
+    # [B]; every part 256-byte aligned
     a = args(num_splits=16)
     rows = 2 * 33 * 64
     order = 256
     o = (16 * rows * 512 * 4 + 255) // 256 * 256
-    l = (16 * rows * 4 + 255) // 256 * 256
+    l = (16 * rows * 4 + 255) // 256 * 256 + 256
     assert lib.va_num_splits(ctypes.byref(a)) == 16
     assert lib.va_workspace_bytes(ctypes.byref(a)) == order + o + l
     assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1))) == order
@@ -197,10 +198,11 @@ def test_fp8_cache_split_planning_and_workspace(lib):
     want = up(pages * 64 * 512 * 2) + up(pages * 64 * 64 * 2) + up(pages * 4)
     assert lib.va_workspace_bytes(ctypes.byref(a)) == 256 + want
     assert lib.va_workspace_bytes(ctypes.byref(args(num_splits=1, dtype=va.VA_F32, **fp8))) == 0
-    # with splits the partials come between the order and the widened cache
+    # with splits the partials and the splits' status come between the order
+    # and the widened cache
     a = args(num_splits=4, **fp8)
     rows = 2 * 33 * 64
-    parts = up(4 * rows * 512 * 4) + up(4 * rows * 4)
+    parts = up(4 * rows * 512 * 4) + up(4 * rows * 4) + up(2 * 4)
     assert lib.va_workspace_bytes(ctypes.byref(a)) == 256 + parts + want
     # the no-allocation entry point refuses, before any launch, what its fixed array cannot hold
     big = args(B=64, max_pages=129, num_splits=1, **fp8)

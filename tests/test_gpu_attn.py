@@ -217,9 +217,12 @@ def test_poisoned_request_stays_contained(va, dtype, path):
 
 
 @pytest.mark.parametrize("dtype,path", [("f32", "f32"), ("bf16", "tc"), ("bf16", "cc")])
-def test_bad_kv_len_and_page_are_flagged(va, dtype, path):
+@pytest.mark.parametrize("num_splits", [1, 3, 0])  # one pass, a split, the planner's choice
+def test_bad_kv_len_and_page_are_flagged(va, dtype, path, num_splits):
+    """A flagged request comes out empty even when only one of its splits
+    meets the bad page."""
     import torch
-    inp = edge_inputs(dtype, B=3, H=8, P=(70, 200), budget=8)
+    inp = edge_inputs(dtype, B=3, H=8, P=(300, 600), budget=8)
     parents = trees_for(inp)["parent"]
     d = to_device(inp, parents)
     mask, _ = va.build_tree_mask(d["parents"])
@@ -230,7 +233,8 @@ def test_bad_kv_len_and_page_are_flagged(va, dtype, path):
     st = torch.zeros(3, dtype=torch.int32, device="cuda")
     flags = va.VA_FLAG_BF16_CUDA_CORES if path == "cc" else 0
     out, lse = va.verify_attn(d["q_nope"], d["q_pe"], d["c_kv"], d["k_pe"], pt, kv, mask,
-                              scale=synth.SCALE, num_splits=1, req_status=st, flags=flags)
+                              scale=synth.SCALE, num_splits=num_splits, req_status=st,
+                              flags=flags)
     torch.cuda.synchronize()
     assert st.cpu().tolist() == [0, va.VA_ERR_INVALID_ARG, va.VA_ERR_INVALID_ARG]
     assert torch.isneginf(lse[1:]).all() and not out[1:].float().abs().sum()
