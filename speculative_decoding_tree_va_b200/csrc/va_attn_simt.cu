@@ -65,7 +65,7 @@ constexpr size_t kSmemTotal = 2 * kSmemK + kSmemSp + kSmemP + 3 * kRows * sizeof
 static_assert(kDqk % (8 * kWarps) == 0, "dims split evenly into float2 steps per lane");
 static_assert(kRows <= kKeys, "the staged Q fits in a key buffer");
 static_assert(kKeys % 8 == 0 && kKeys / 8 <= 8, "8-key groups in Q.K^T; 8 softmax lanes per row");
-static_assert(kKeys == 32, "bulk staging: one key row per lane of one warp");
+static_assert(kKeys == 32, "bulk staging: lanes 0-7 of warp 0 copy 4 c_kv rows each");
 static_assert(kRows == kKeys, "the staged Q uses the tile layout");
 static_assert(kDc == 64 * kWarps && kDr == 8 * kWarps && kSub == 18,
               "per warp: 64 c_kv columns and 8 k_pe columns, 8 + 1 pairs per lane");
