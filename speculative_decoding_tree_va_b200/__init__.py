@@ -199,6 +199,8 @@ def workspace_bytes(args: VaAttnArgs) -> int:
 
 
 def num_splits(args: VaAttnArgs) -> int:
+    """The split count va_verify_attn uses for these arguments (for the balanced
+    CUDA-core plan, the number of partials per row it merges)."""
     return int(load_library().va_num_splits(ctypes.byref(args)))
 
 
