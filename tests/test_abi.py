@@ -175,6 +175,37 @@ def test_balanced_cuda_core_plan(lib, B, T, H, max_pages):
     assert tc >= 1 and (tc & (tc - 1)) == 0  # the power-of-two planner
 
 
+def test_balanced_cta_of_is_the_inverse_of_the_ranges():
+    """The balanced plan's kernel finds a segment's first and last CTA (its
+    partial slots, and who marks the unused ones) with
+    cta_of(u) = floor((u G + G - 1) / U), the CTA whose range
+    [c U / G, (c + 1) U / G) holds virtual tile u.  Checked against the ranges
+    themselves: every tile has exactly one owner, a segment's owners are
+    consecutive CTAs from cta_of(first tile) to cta_of(last tile), and so slot
+    c - cta_of(first) is unique per segment and below the plan's slot count."""
+    import random
+    rng = random.Random(7)
+    cta_of = lambda u, U, G: (u * G + G - 1) // U
+    for _ in range(300):
+        q = rng.randint(1, 40)
+        vt = rng.randint(1, 300)
+        U = q * vt
+        G = rng.randint(q + 1, max(q + 1, min(148, U // 4 if U >= 4 * (q + 1) else q + 1)))
+        owner = [None] * U
+        for c in range(G):
+            for u in range(c * U // G, (c + 1) * U // G):
+                assert owner[u] is None
+                owner[u] = c
+        assert None not in owner
+        for u in range(U):
+            assert cta_of(u, U, G) == owner[u], (u, U, G)
+        for seg in range(q):
+            owners = sorted({owner[u] for u in range(seg * vt, (seg + 1) * vt)})
+            assert owners == list(range(owners[0], owners[-1] + 1))
+            assert owners[0] == cta_of(seg * vt, U, G)
+            assert owners[-1] == cta_of((seg + 1) * vt - 1, U, G)
+
+
 def test_fp8_cache_split_planning_and_workspace(lib):
     """An FP8 cache keeps the query type's kernel (bf16: tensor cores, fp32: CUDA
     cores), so the auto split count is that kernel's; bf16 on the tensor cores
