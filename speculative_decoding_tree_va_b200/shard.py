@@ -20,6 +20,12 @@ them.
 The steps are plain functions of callables so that the rank plumbing runs on
 CPU ranks (``gloo``) in the tests; ``ShardedStep`` binds them to the CUDA
 library and NCCL.
+
+Problems a split meets (a bad kv_len or page index, an expired wait) are
+reported by each rank's partials call in that rank's ``req_status``; the
+final merge does not see them, so a request flagged on any rank is to be
+treated as failed (its merged rows are not emptied across ranks, unlike a
+one-GPU split call, whose merge empties them).
 """
 from __future__ import annotations
 
