@@ -720,13 +720,13 @@ def run_reference(args):
     flops, alg_bytes = work(inp, depth)
     ms = flops / (v * 1e12) * 1e3
     S = args.splits if getattr(args, "splits", None) is not None else wl.splits
-    cfg = config_of(wl, S, args.gpus, flops, alg_bytes)
-    cfg["note"] = "each step = a bounded row sample; per-step time extrapolated per flop"
+    cfg = config_of(wl, S, args.gpus, flops, alg_bytes)  # the native arm's config, unchanged
     line = {
         "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; no dataset or weights)", "impl": "reference",
+        "note": "each step = a bounded row sample; per-step time extrapolated per flop",
         "config": cfg,
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                          "sample": vals[0]["sample"], "host": vals[0]["host"]},
